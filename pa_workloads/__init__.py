@@ -1,0 +1,272 @@
+"""Seeded synthetic inputs for the paged decode attention workloads.
+
+This module draws numbers and nothing else: sequence lengths, the pool's
+initial free-list order, token ids for prefix hashing, N(0,1) query/key/value
+values cast to the input dtype, and per-tensor FP8 scales from the drawn
+values' absolute maximum.  It holds none of the method's arithmetic (no block
+tables, slots, cache writes or attention); the oracle and the CUDA path each
+derive those from these same arrays.
+
+Workloads (sizes as named by the paged-attention benchmark plan):
+
+* ``tiny_fp32``: 4 sequences, context [40,128,300,64], block 16, a pool of
+  128 blocks handed out in a seeded random permutation, 2 query = 2 KV heads,
+  head_dim 64, fp32 N(0,1) seed 0; one decode step.
+* ``gqa_bf16``: 64 sequences, context uniform in [32, 2048], 32 query / 8 KV
+  heads, head_dim 128, block 16, pool 1.25x the blocks needed, shuffled.
+* ``prefix_bf16``: 256 sequences; half share one 1024-token prefix (64
+  blocks); suffix lengths lognormal (median 512, sigma 1) clipped to
+  [16, 8192]; 32/8 heads, head_dim 128, block 16.
+* ``fp8_long``: 128 sequences, context uniform in [4096, 32768], 64/8 heads,
+  head_dim 128, block 16, FP8-e4m3 cache with per-tensor K and V scales,
+  bf16 queries and bf16 new K/V.
+* ``mixed_prefill``: 8 prefill chunks of 512 query tokens over 0..4096 prior
+  tokens each, plus 248 decode rows over contexts uniform in [64, 4096];
+  32/8 heads, head_dim 128, block 16 or 32.
+
+Each has a ``small`` variant with the same structure at sizes a plain CPU
+oracle finishes in seconds.  Randomness: ``tiny_fp32`` draws everything from
+``np.random.default_rng(0)`` in a fixed order (permutation, then per sequence
+K then V, then new K, new V, q); the others use one independent stream per
+(workload, sequence, purpose) via ``np.random.SeedSequence``.
+"""
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+import torch
+
+GLOBAL = 2**31 - 1  # sequence index used by per-workload streams
+
+S_LENGTHS, S_PERM, S_K, S_V, S_KNEW, S_VNEW, S_Q, S_TOKENS, S_SUFFIX = range(9)
+
+DTYPE_TORCH = {"f32": torch.float32, "bf16": torch.bfloat16}
+FP8_MAX = 448.0
+
+
+def rng(seed_key: int, seq: int, stream: int) -> np.random.Generator:
+    return np.random.default_rng(np.random.SeedSequence([0, int(seed_key), int(seq), int(stream)]))
+
+
+def _cast(x: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t if dtype == "f32" else t.to(DTYPE_TORCH[dtype])
+
+
+@dataclass
+class Workload:
+    name: str
+    seed_key: int
+    kv_dtype: str  # storage of the cache: "f32" | "bf16" | "e4m3"
+    q_dtype: str  # queries and new K/V: "f32" | "bf16"
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    context_lens: np.ndarray  # int64 [S]: tokens cached before the step
+    q_lens: np.ndarray  # int64 [S]: tokens added this step (1 = decode row)
+    free_order: np.ndarray  # int32 [num_blocks]: initial free-list order
+    prefix_len: int = 0
+    sharing: Optional[np.ndarray] = None  # bool [S]
+    vocab: int = 32000
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+    _fixed: Optional[dict] = field(default=None, repr=False)
+
+    # ---- shape helpers (no method arithmetic) --------------------------------
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def num_new_tokens(self) -> int:
+        return int(self.q_lens.sum())
+
+    @property
+    def max_q_len(self) -> int:
+        return int(self.q_lens.max()) if self.num_seqs else 0
+
+    # ---- draws ---------------------------------------------------------------
+    def token_ids(self, s: int) -> Optional[np.ndarray]:
+        """Token ids of the cached context of sequence s (None: no hashing)."""
+        if self.sharing is None:
+            return None
+        n = int(self.context_lens[s])
+        own = rng(self.seed_key, s, S_TOKENS).integers(0, self.vocab, size=n, dtype=np.int64)
+        if self.sharing[s]:
+            pre = rng(self.seed_key, GLOBAL, S_TOKENS).integers(0, self.vocab, size=self.prefix_len,
+                                                                dtype=np.int64)
+            own[: self.prefix_len] = pre
+        return own.astype(np.int32)
+
+    def _normal(self, seq: int, stream: int, rows: int, heads: int) -> np.ndarray:
+        return rng(self.seed_key, seq, stream).standard_normal((rows, heads, self.head_dim),
+                                                               dtype=np.float32)
+
+    def prior_kv_f32(self, s: int):
+        """fp32 draws of K and V for the cached context of sequence s:
+        [context_len][kv_heads][head_dim] each."""
+        if self._fixed is not None:
+            return self._fixed["k"][s], self._fixed["v"][s]
+        n = int(self.context_lens[s])
+        k = self._normal(s, S_K, n, self.num_kv_heads)
+        v = self._normal(s, S_V, n, self.num_kv_heads)
+        if self.sharing is not None and self.sharing[s]:
+            p = self.prefix_len
+            k[:p] = self._normal(GLOBAL, S_K, p, self.num_kv_heads)
+            v[:p] = self._normal(GLOBAL, S_V, p, self.num_kv_heads)
+        return k, v
+
+    def prior_kv(self, s: int):
+        """K, V of sequence s's cached context in the input dtype (torch, CPU)."""
+        k, v = self.prior_kv_f32(s)
+        return _cast(k, self.q_dtype), _cast(v, self.q_dtype)
+
+    def new_kv(self):
+        """K, V of this step's new tokens: [num_new_tokens][kv_heads][head_dim]."""
+        if self._fixed is not None:
+            return _cast(self._fixed["k_new"], self.q_dtype), _cast(self._fixed["v_new"], self.q_dtype)
+        t = self.num_new_tokens
+        k = self._normal(GLOBAL, S_KNEW, t, self.num_kv_heads)
+        v = self._normal(GLOBAL, S_VNEW, t, self.num_kv_heads)
+        return _cast(k, self.q_dtype), _cast(v, self.q_dtype)
+
+    def queries(self):
+        """Queries of this step's new tokens: [num_new_tokens][q_heads][head_dim]."""
+        if self._fixed is not None:
+            return _cast(self._fixed["q"], self.q_dtype)
+        return _cast(self._normal(GLOBAL, S_Q, self.num_new_tokens, self.num_q_heads), self.q_dtype)
+
+    def set_fp8_scales(self, amax_k: float, amax_v: float):
+        """Per-tensor scales = amax / 448 (fp32), so the largest drawn value
+        maps onto the largest finite e4m3 value."""
+        self.k_scale = float(np.float32(amax_k) / np.float32(FP8_MAX))
+        self.v_scale = float(np.float32(amax_v) / np.float32(FP8_MAX))
+
+    def fp8_scales_from_draws(self):
+        """amax over every K (V) value this workload draws, prior and new, in
+        the input dtype; sets and returns (k_scale, v_scale)."""
+        ak = av = 0.0
+        for s in range(self.num_seqs):
+            k, v = self.prior_kv(s)
+            if k.numel():
+                ak = max(ak, float(k.abs().max()))
+                av = max(av, float(v.abs().max()))
+        k, v = self.new_kv()
+        if k.numel():
+            ak = max(ak, float(k.abs().max()))
+            av = max(av, float(v.abs().max()))
+        self.set_fp8_scales(ak, av)
+        return self.k_scale, self.v_scale
+
+
+def _pool_size(need_blocks: int) -> int:
+    return int(np.ceil(1.25 * need_blocks))
+
+
+def _blocks_needed(context_lens, q_lens, bs, shared_blocks=0, n_sharing=0):
+    # capacity bookkeeping for sizing the pool only: whole blocks per sequence
+    tot = sum(-(-(int(c) + int(q)) // bs) for c, q in zip(context_lens, q_lens))
+    return tot - shared_blocks * max(0, n_sharing - 1)
+
+
+def _finish(name, seed_key, kv_dtype, q_dtype, hq, hkv, d, bs, ctx, qlen, nb=None,
+            prefix_len=0, sharing=None) -> Workload:
+    ctx = np.asarray(ctx, dtype=np.int64)
+    qlen = np.asarray(qlen, dtype=np.int64)
+    if nb is None:
+        shared_blocks = prefix_len // bs
+        n_sharing = int(sharing.sum()) if sharing is not None else 0
+        nb = _pool_size(_blocks_needed(ctx, qlen, bs, shared_blocks, n_sharing))
+        nb = max(nb, 1)
+    order = rng(seed_key, GLOBAL, S_PERM).permutation(nb).astype(np.int32)
+    return Workload(name, seed_key, kv_dtype, q_dtype, hq, hkv, d, bs, nb, ctx, qlen, order,
+                    prefix_len, sharing)
+
+
+def tiny_fp32() -> Workload:
+    lens = [40, 128, 300, 64]
+    hq = hkv = 2
+    d = 64
+    g = np.random.default_rng(0)
+    perm = g.permutation(128).astype(np.int32)
+    ks, vs = [], []
+    for n in lens:
+        ks.append(g.standard_normal((n, hkv, d), dtype=np.float32))
+        vs.append(g.standard_normal((n, hkv, d), dtype=np.float32))
+    k_new = g.standard_normal((4, hkv, d), dtype=np.float32)
+    v_new = g.standard_normal((4, hkv, d), dtype=np.float32)
+    q = g.standard_normal((4, hq, d), dtype=np.float32)
+    return Workload("tiny_fp32", 0, "f32", "f32", hq, hkv, d, 16, 128,
+                    np.array(lens, dtype=np.int64), np.ones(4, dtype=np.int64), perm,
+                    _fixed={"k": ks, "v": vs, "k_new": k_new, "v_new": v_new, "q": q})
+
+
+def gqa_bf16(size: str = "full") -> Workload:
+    key = 1 if size == "full" else 101
+    n, lo, hi = (64, 32, 2048) if size == "full" else (6, 0, 300)
+    ctx = rng(key, GLOBAL, S_LENGTHS).integers(lo, hi, size=n, endpoint=True)
+    return _finish("gqa_bf16" + ("" if size == "full" else "_small"), key, "bf16", "bf16",
+                   32, 8, 128, 16, ctx, np.ones(n))
+
+
+def prefix_bf16(size: str = "full") -> Workload:
+    key = 2 if size == "full" else 102
+    if size == "full":
+        n, prefix, median, lo, hi = 256, 1024, 512, 16, 8192
+    else:
+        n, prefix, median, lo, hi = 8, 64, 40, 16, 200
+    suf = rng(key, GLOBAL, S_SUFFIX).lognormal(mean=np.log(median), sigma=1.0, size=n)
+    suf = np.clip(np.rint(suf), lo, hi).astype(np.int64)
+    sharing = np.zeros(n, dtype=bool)
+    sharing[: n // 2] = True
+    ctx = suf + np.where(sharing, prefix, 0)
+    return _finish("prefix_bf16" + ("" if size == "full" else "_small"), key, "bf16", "bf16",
+                   32, 8, 128, 16, ctx, np.ones(n), prefix_len=prefix, sharing=sharing)
+
+
+def fp8_long(size: str = "full") -> Workload:
+    key = 3 if size == "full" else 103
+    n, lo, hi = (128, 4096, 32768) if size == "full" else (4, 100, 700)
+    ctx = rng(key, GLOBAL, S_LENGTHS).integers(lo, hi, size=n, endpoint=True)
+    return _finish("fp8_long" + ("" if size == "full" else "_small"), key, "e4m3", "bf16",
+                   64, 8, 128, 16, ctx, np.ones(n))
+
+
+def mixed_prefill(block_size: int = 16, size: str = "full") -> Workload:
+    key = 4 if size == "full" else 104
+    if size == "full":
+        nchunk, chunk, plo, phi, ndec, dlo, dhi = 8, 512, 0, 4096, 248, 64, 4096
+    else:
+        nchunk, chunk, plo, phi, ndec, dlo, dhi = 2, 40, 0, 100, 5, 10, 200
+    g = rng(key, GLOBAL, S_LENGTHS)
+    pre = g.integers(plo, phi, size=nchunk, endpoint=True)
+    dec = g.integers(dlo, dhi, size=ndec, endpoint=True)
+    ctx = np.concatenate([pre, dec])
+    qlen = np.concatenate([np.full(nchunk, chunk), np.ones(ndec)])
+    return _finish(f"mixed_prefill_bs{block_size}" + ("" if size == "full" else "_small"), key,
+                   "bf16", "bf16", 32, 8, 128, block_size, ctx, qlen)
+
+
+def custom(name, context_lens, q_lens=None, kv_dtype="bf16", q_dtype="bf16", num_q_heads=8,
+           num_kv_heads=2, head_dim=128, block_size=16, seed_key=900, num_blocks=None) -> Workload:
+    """Explicit shapes for edge-case tests."""
+    ctx = np.asarray(context_lens, dtype=np.int64)
+    ql = np.ones_like(ctx) if q_lens is None else np.asarray(q_lens, dtype=np.int64)
+    return _finish(name, seed_key, kv_dtype, q_dtype, num_q_heads, num_kv_heads, head_dim,
+                   block_size, ctx, ql, nb=num_blocks)
+
+
+WORKLOADS = {
+    "tiny_fp32": lambda size="full": tiny_fp32(),
+    "gqa_bf16": gqa_bf16,
+    "prefix_bf16": prefix_bf16,
+    "fp8_long": fp8_long,
+    "mixed_prefill_bs16": lambda size="full": mixed_prefill(16, size),
+    "mixed_prefill_bs32": lambda size="full": mixed_prefill(32, size),
+}
+
+
+def make(name: str, size: str = "full") -> Workload:
+    return WORKLOADS[name](size)
