@@ -79,16 +79,25 @@ def e4m3_encode(x) -> np.ndarray:
     return np.array([f(float(v)) for v in x.ravel()], dtype=np.uint8).reshape(x.shape)
 
 
-def new_cache(num_blocks, num_kv_heads, block_size, head_dim, kv_dtype):
-    """A K or V pool [NB][Hkv][bs][D] in the device's storage format, filled
-    with a sentinel (NaN for fp32/bf16, the e4m3 NaN code for fp8) so that any
-    read of an unwritten slot shows up."""
-    shape = (num_blocks, num_kv_heads, block_size, head_dim)
+def new_cache(num_blocks, num_kv_heads, block_size, head_dim, kv_dtype, d_major=False):
+    """A K or V pool in the storage format, filled with a sentinel (NaN for
+    fp32/bf16, the e4m3 NaN code for fp8) so that any read of an unwritten
+    slot shows up.  Token-major [NB][Hkv][bs][D]; d_major=True gives
+    [NB][Hkv][D][bs], the layout of an e4m3 V pool."""
+    shape = (num_blocks, num_kv_heads, head_dim, block_size) if d_major else \
+        (num_blocks, num_kv_heads, block_size, head_dim)
     if kv_dtype == "f32":
         return np.full(shape, np.nan, dtype=np.float32)
     if kv_dtype == "bf16":
         return np.full(shape, 0x7FC0, dtype=np.uint16)
     return np.full(shape, 0x7F, dtype=np.uint8)
+
+
+def new_caches(num_blocks, num_kv_heads, block_size, head_dim, kv_dtype):
+    """(K pool, V pool) in the layouts the cache write uses for kv_dtype."""
+    return (new_cache(num_blocks, num_kv_heads, block_size, head_dim, kv_dtype),
+            new_cache(num_blocks, num_kv_heads, block_size, head_dim, kv_dtype,
+                      d_major=(kv_dtype == "e4m3")))
 
 
 def cache_write(k_new, v_new, slot_mapping, k_cache, v_cache, in_dtype, kv_dtype,
@@ -97,12 +106,15 @@ def cache_write(k_new, v_new, slot_mapping, k_cache, v_cache, in_dtype, kv_dtype
 
     k_new, v_new: [T][Hkv][D] raw storage (float32 array for fp32, uint16 bits
     for bf16).  slot_mapping: int64 [T]; a negative slot is skipped.
+    k_cache is [NB][Hkv][bs][D]; v_cache is too, except for e4m3 where it is
+    d-major [NB][Hkv][D][bs].
     """
     k_new = np.ascontiguousarray(k_new)
     v_new = np.ascontiguousarray(v_new)
     slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
     nb, hkv, bs, d = k_cache.shape
     assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    assert v_cache.shape == ((nb, hkv, d, bs) if kv_dtype == "e4m3" else (nb, hkv, bs, d))
     assert k_new.shape == (slots.shape[0], hkv, d), k_new.shape
     assert k_new.dtype == _NPDT[in_dtype] and k_cache.dtype == _NPDT[kv_dtype]
     rc = lib().oracle_cache_write(_DT[in_dtype], _DT[kv_dtype], _ptr(k_new), _ptr(v_new),
@@ -129,6 +141,7 @@ def attention(q, row_seq, row_pos, block_tables, k_cache, v_cache, kv_dtype, num
     row_pos = np.ascontiguousarray(row_pos, dtype=np.int32)
     bt = np.ascontiguousarray(block_tables, dtype=np.int32)
     nb, hkv, bs, d = k_cache.shape
+    assert v_cache.shape == ((nb, hkv, d, bs) if kv_dtype == "e4m3" else (nb, hkv, bs, d))
     r = q.shape[0]
     assert q.shape == (r, num_q_heads, d)
     out = np.empty((r, num_q_heads, d), dtype=np.float64)

@@ -25,6 +25,12 @@
  *    block table[j / bs] at offset j % bs.  Straight loops, fp64 throughout,
  *    no online softmax, no blocking.
  *
+ *  - Cache layout (the pages leave it open; this is the build's reading):
+ *    K is [num_blocks][kv_heads][block_size][head_dim] for every dtype; V is
+ *    the same for fp32/bf16 caches, and d-major [num_blocks][kv_heads]
+ *    [head_dim][block_size] for e4m3 caches.  The index of element d of the
+ *    token at offset o of block b, head h, is written out at each use.
+ *
  *  - e4m3 encode/decode from the OCP 8-bit floating point definition (E4M3:
  *    sign, 4 exponent bits with bias 7, 3 mantissa bits, exponent field 0 is
  *    subnormal, S.1111.111 is NaN, no infinities, largest finite 448).
@@ -114,8 +120,16 @@ static double orc_load_cache(const void* p, int dt, size_t i, double scale) {
 
 /* ---- cache write -------------------------------------------------------- */
 
+/* Offset of element d of the token at (block b, head h, offset o): token-major
+ * [b][h][o][d], or d-major [b][h][d][o] (e4m3 V). */
+static size_t orc_index(int d_major, size_t b, size_t h, size_t o, size_t d, int num_kv_heads,
+                        int block_size, int head_dim) {
+  if (d_major) return ((b * num_kv_heads + h) * head_dim + d) * block_size + o;
+  return ((b * num_kv_heads + h) * block_size + o) * head_dim + d;
+}
+
 /* k_new, v_new: [num_tokens][num_kv_heads][head_dim] in in_dtype (fp32 or bf16).
- * k_cache, v_cache: [num_blocks][num_kv_heads][block_size][head_dim] in kv_dtype.
+ * k_cache, v_cache: the pools, laid out as described at the top of this file.
  * A negative slot is skipped.  Returns 0, or -1 if a slot is past the pool. */
 int oracle_cache_write(int in_dtype, int kv_dtype, const void* k_new, const void* v_new,
                        const int64_t* slots, int num_tokens, int num_blocks, int block_size,
@@ -136,7 +150,9 @@ int oracle_cache_write(int in_dtype, int kv_dtype, const void* k_new, const void
       for (h = 0; h < num_kv_heads; ++h) {
         for (d = 0; d < head_dim; ++d) {
           size_t si = ((size_t)t * num_kv_heads + h) * head_dim + d;
-          size_t di = (((size_t)blk * num_kv_heads + h) * block_size + off) * head_dim + d;
+          int d_major = (side == 1 && kv_dtype == ORC_E4M3);
+          size_t di = orc_index(d_major, (size_t)blk, (size_t)h, (size_t)off, (size_t)d, num_kv_heads,
+                                block_size, head_dim);
           if (kv_dtype == ORC_E4M3) {
             float x = orc_load_f32(src, in_dtype, si);
             float y = x / scale; /* one IEEE fp32 division */
@@ -186,9 +202,11 @@ void oracle_attention(const double* q, int num_rows, const int32_t* row_seq, con
     for (j = 0; j < n; ++j) {
       int32_t blk = block_tables[(size_t)s * max_blocks + j / block_size];
       int off = j % block_size;
-      size_t base = (((size_t)blk * num_kv_heads + kvh) * block_size + off) * head_dim;
       double dot = 0.0;
-      for (d = 0; d < head_dim; ++d) dot += qv[d] * orc_load_cache(k_cache, kv_dtype, base + d, k_scale);
+      for (d = 0; d < head_dim; ++d)
+        dot += qv[d] * orc_load_cache(k_cache, kv_dtype,
+                                      orc_index(0, blk, kvh, off, d, num_kv_heads, block_size, head_dim),
+                                      k_scale);
       logit[j] = scale * dot;
       if (logit[j] > mx) mx = logit[j];
     }
@@ -197,9 +215,12 @@ void oracle_attention(const double* q, int num_rows, const int32_t* row_seq, con
     for (j = 0; j < n; ++j) {
       int32_t blk = block_tables[(size_t)s * max_blocks + j / block_size];
       int off = j % block_size;
-      size_t base = (((size_t)blk * num_kv_heads + kvh) * block_size + off) * head_dim;
       double w = exp(logit[j] - mx) / z;
-      for (d = 0; d < head_dim; ++d) o[d] += w * orc_load_cache(v_cache, kv_dtype, base + d, v_scale);
+      for (d = 0; d < head_dim; ++d)
+        o[d] += w * orc_load_cache(v_cache, kv_dtype,
+                                   orc_index(kv_dtype == ORC_E4M3, blk, kvh, off, d, num_kv_heads,
+                                             block_size, head_dim),
+                                   v_scale);
     }
     free(logit);
   }

@@ -128,8 +128,7 @@ def test_cache_write_fp8_matches_torch_quantisation():
     v = torch.from_numpy(3 * g.standard_normal((40, hkv, d), dtype=np.float32)).bfloat16()
     ks = float(np.float32(k.abs().max().item()) / np.float32(448))
     vs = float(np.float32(v.abs().max().item()) / np.float32(448))
-    kc = oracle.new_cache(nb, hkv, bs, d, "e4m3")
-    vc = oracle.new_cache(nb, hkv, bs, d, "e4m3")
+    kc, vc = oracle.new_caches(nb, hkv, bs, d, "e4m3")
     slots = g.permutation(nb * bs)[:40]
     oracle.cache_write(k.view(torch.int16).numpy().view(np.uint16),
                        v.view(torch.int16).numpy().view(np.uint16), slots, kc, vc, "bf16", "e4m3",
@@ -138,7 +137,19 @@ def test_cache_write_fp8_matches_torch_quantisation():
     vq = (v.float() / torch.tensor(vs, dtype=torch.float32)).to(E4M3).view(torch.uint8).numpy()
     for t, s in enumerate(slots):
         assert np.array_equal(kc[s // bs, :, s % bs], kq[t])
-        assert np.array_equal(vc[s // bs, :, s % bs], vq[t])
+        assert np.array_equal(vc[s // bs, :, :, s % bs], vq[t])  # V is d-major for e4m3
+
+
+def test_cache_write_fp8_v_is_d_major_by_hand():
+    nb, hkv, bs, d = 2, 1, 4, 3
+    kc, vc = oracle.new_caches(nb, hkv, bs, d, "e4m3")
+    k = np.array([[[1.0, 2.0, 3.0]]], dtype=np.float32)
+    oracle.cache_write(k, -k, np.array([6]), kc, vc, "f32", "e4m3", 1.0, 1.0)
+    flat_v = vc.ravel()
+    # slot 6 -> block 1, offset 2; element d sits at ((1*1+0)*3 + d)*4 + 2
+    assert [flat_v[(3 + dd) * 4 + 2] for dd in range(3)] == [0xB8, 0xC0, 0xC4]  # -1, -2, -3
+    assert [kc.ravel()[(1 * 4 + 2) * 3 + dd] for dd in range(3)] == [0x38, 0x40, 0x44]
+    assert (flat_v == 0x7F).sum() == flat_v.size - 3
 
 
 # ---------------------------------------------------------------- attention
@@ -157,8 +168,7 @@ def _paged_problem(lens, hq, hkv, d, bs, kv_dtype="f32", seed=0, shuffle=True, q
         pos += m
     ks = [g.standard_normal((n, hkv, d)).astype(np.float32) for n in lens]
     vs = [g.standard_normal((n, hkv, d)).astype(np.float32) for n in lens]
-    kc = oracle.new_cache(nb, hkv, bs, d, kv_dtype)
-    vc = oracle.new_cache(nb, hkv, bs, d, kv_dtype)
+    kc, vc = oracle.new_caches(nb, hkv, bs, d, kv_dtype)
     for s, n in enumerate(lens):
         slots = np.array([tables[s, p // bs] * bs + p % bs for p in range(n)], dtype=np.int64)
         oracle.cache_write(ks[s], vs[s], slots, kc, vc, "f32", kv_dtype)
@@ -261,8 +271,7 @@ def test_fp8_attention_uses_dequantised_values():
     # requantise the cache to e4m3 with scales, then compare with SDPA on the
     # values torch decodes from the same codes
     ks, vs = 0.01, 0.02
-    kc = oracle.new_cache(*P["kc"].shape, "e4m3")
-    vc = oracle.new_cache(*P["vc"].shape, "e4m3")
+    kc, vc = oracle.new_caches(*P["kc"].shape, "e4m3")
     for s, n in enumerate(lens):
         slots = np.array([P["tables"][s, p // bs] * bs + p % bs for p in range(n)])
         oracle.cache_write(P["ks"][s], P["vs"][s], slots, kc, vc, "f32", "e4m3", ks, vs)
@@ -271,6 +280,6 @@ def test_fp8_attention_uses_dequantised_values():
     for s, n in enumerate(lens):
         slots = [P["tables"][s, p // bs] * bs + p % bs for p in range(n)]
         kd = np.stack([_torch_e4m3_value(kc[x // bs, :, x % bs]) for x in slots]) * np.float64(np.float32(ks))
-        vd = np.stack([_torch_e4m3_value(vc[x // bs, :, x % bs]) for x in slots]) * np.float64(np.float32(vs))
+        vd = np.stack([_torch_e4m3_value(vc[x // bs, :, :, x % bs]) for x in slots]) * np.float64(np.float32(vs))
         ref = _sdpa(q[s], kd, vd, 0.25, hq, hkv, n - 1)
         np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
