@@ -1,0 +1,330 @@
+"""Benchmark: one attention layer-step of paged decode (pa_cache_write of the
+step's new K/V + pa_decode) on a seeded synthetic batch, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is KV GB/s: the step's algorithmic
+attention bytes (every valid token's K and V once, shared prefix blocks
+once, plus queries, outputs, table entries and lengths) divided by the step
+time, summed over all ranks (replicas: the path has no cross-GPU exchange).
+`--impl reference` times the CPU oracle on this host's cores instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import pa_workloads as W  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s"
+DEFAULT_WORKLOAD = "gqa_bf16"
+KV_BYTES = {"f32": 4, "bf16": 2, "e4m3": 1}
+Q_BYTES = {"f32": 4, "bf16": 2}
+
+
+def algorithmic_bytes(wl):
+    """Bytes the attention of one step must move at least once (HBM)."""
+    bs, hkv, d = wl.block_size, wl.num_kv_heads, wl.head_dim
+    seq_lens = wl.context_lens + wl.q_lens
+    tokens = int(seq_lens.sum())
+    if wl.sharing is not None:  # the shared prefix is stored (and read) once
+        tokens -= wl.prefix_len * max(0, int(wl.sharing.sum()) - 1)
+    kv = tokens * 2 * hkv * d * KV_BYTES[wl.kv_dtype]
+    rows = wl.num_new_tokens
+    qo = 2 * rows * wl.num_q_heads * d * Q_BYTES[wl.q_dtype]
+    table = int(sum(-(-int(n) // bs) for n in seq_lens)) * 4 + 4 * wl.num_seqs
+    return kv + qo + table, kv
+
+
+def logical_kv_bytes(wl):
+    seq_lens = wl.context_lens + wl.q_lens
+    return int(seq_lens.sum()) * 2 * wl.num_kv_heads * wl.head_dim * KV_BYTES[wl.kv_dtype]
+
+
+def write_bytes(wl):
+    t = wl.num_new_tokens
+    return t * wl.num_kv_heads * wl.head_dim * 2 * (Q_BYTES[wl.q_dtype] + KV_BYTES[wl.kv_dtype]) + 8 * t
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons while the timed region runs."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                             timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def oracle_prepare(wl, seqs):
+    from oracle.workload import prepare  # test infrastructure: the CPU baseline only
+    return prepare(wl, seqs)
+
+
+def oracle_time(prep):
+    """Wall time of the oracle's own arithmetic (cache writes + attention) on
+    a prepared sample; the draws and pool replay are prepared beforehand."""
+    from oracle.workload import compute
+    t0 = time.perf_counter()
+    compute(prep)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(wl, budget_s):
+    """A prefix of the batch whose oracle evaluation takes about budget_s
+    (scaled from a timing of the first sequence); its KV bytes."""
+    import oracle
+    t = oracle_time(oracle_prepare(wl, [0]))
+    per_token = t / max(1, int(wl.context_lens[0] + wl.q_lens[0]))
+    seqs, est = [], 0.0
+    for s in range(wl.num_seqs):
+        n = int(wl.context_lens[s] + wl.q_lens[s])
+        if seqs and est + per_token * n > budget_s:
+            break
+        seqs.append(s)
+        est += per_token * n
+    kv = sum(int(wl.context_lens[s] + wl.q_lens[s]) for s in seqs) * 2 * wl.num_kv_heads * wl.head_dim * \
+        KV_BYTES[wl.kv_dtype]
+    return oracle_prepare(wl, seqs), len(seqs), kv, oracle.max_threads()
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    prep, n, kv, cores = oracle_sample(wl, budget_s)
+    t = oracle_time(prep)
+    return {"value": kv / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {wl.num_seqs} sequences of {wl.name}: their cache writes and all their "
+                      f"query rows, fp64 C oracle, {t:.2f} s"}
+
+
+def bench_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    wl = W.make(args.workload, "full")
+    if wl.kv_dtype == "e4m3":
+        wl.fp8_scales_from_draws()
+    per_step = max(0.05, min(args.ref_budget, 150.0 / (args.steps + args.warmup)))
+    prep, n, kv, cores = oracle_sample(wl, per_step)
+    for _ in range(args.warmup):
+        oracle_time(prep)
+    times = [oracle_time(prep) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = kv / t / 1e9
+    sample = f"{n} of {wl.num_seqs} sequences of {wl.name} per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "sample_seqs": n},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def bench_ours(args):
+    world, rank, local = dist_setup(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import paged_kv_cache_452_b200 as pa
+    from paged_kv_cache_452_b200 import runner
+
+    wl = W.make(args.workload, "full")
+    # two copies of the pool, used alternately, so no step finds the previous
+    # step's K/V in L2 (each copy is larger than L2 already)
+    batches = [runner.setup(wl, device) for _ in range(2)]
+    alg_bytes, kv_bytes = algorithmic_bytes(wl)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        runner.step(batches[i & 1])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.2 if sampler else 0)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, device)
+
+    # the dominant call, pa_decode (decode kernel + its log-sum-exp combine),
+    # timed per launch with events on its stream over the same number of steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        runner.write_step(batches[i & 1])
+        evs[i][0].record(stream)
+        runner.attend(batches[i & 1])
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    attend_ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world, device)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, write + decode, D2H of the output
+    b0 = batches[0]
+    host = {k: getattr(b0, k).cpu().pin_memory() for k in ("q", "k_new", "v_new", "slots", "tables", "seq_lens")}
+    out_host = torch.empty(b0.out.shape, dtype=b0.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    for i in range(max(1, args.warmup)):
+        for k, t in host.items():
+            getattr(b0, k).copy_(t, non_blocking=True)
+        runner.step(b0)
+        out_host.copy_(b0.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        for k, t in host.items():
+            getattr(b0, k).copy_(t, non_blocking=True)
+        runner.step(b0)
+        out_host.copy_(b0.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, device)
+
+    errs = [pa.workspace_error(b.workspace) for b in batches]
+    if any(errs):
+        raise SystemExit(f"kernel error word set: {errs}")
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    peaks, src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    achieved = alg_bytes / (attend_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": world * alg_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.kv_dtype if wl.kv_dtype != "e4m3" else "fp8_e4m3",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": wl.block_size,
+                   "context_tokens": int((wl.context_lens + wl.q_lens).sum()), "kv_bytes": kv_bytes,
+                   "algorithmic_bytes": alg_bytes, "parallelism": f"replicas x{world}",
+                   "l2": "2 pool copies used alternately, each larger than L2"},
+        "decode_tokens_per_s": world * wl.num_seqs / (ms * 1e-3),
+        "fraction_of_8tbs": world * alg_bytes / (ms * 1e-3) / 1e9 / 8000.0 / world,
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_tc_kernel + decode_combine_kernel)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": src, "traffic": None, "pa_decode_ms": attend_ms},
+        "e2e": {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.ref_budget)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

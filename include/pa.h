@@ -1,0 +1,221 @@
+/*
+ * pa.h -- C ABI of the paged KV-cache decode-attention library (libpa.so).
+ *
+ * The operation.  A sequence's keys and values live in fixed-size physical
+ * blocks of block_size tokens (16 by default) drawn from one pool; the blocks
+ * of a sequence need not be contiguous, and a per-sequence block table maps
+ * its logical block i to a physical block ("vLLM innenfra: slik gjør paged
+ * attention GPU-minnet til blokker på 16 tokens", paragraph 2; "49 vLLM /
+ * PagedAttention", section "Идея и механизм"; "PagedAttention：KV cache 即虚拟
+ * 内存（block manager & 碎片）", section 直接答案).  Paging changes neither
+ * the attention output nor the amount of compute (same page, follow-up
+ * "分页改变输出或加速 kernel 吗？"): the kernels here compute ordinary softmax
+ * attention, gathering K/V through the table.
+ *
+ * Conventions for every call
+ *  - Return value: PA_OK (0) or a pa_status error code; pa_last_error()
+ *    returns a message for the last failure on the calling thread.
+ *  - Device pointers are owned by the caller.  The library never allocates
+ *    device memory: scratch space comes from a caller buffer sized by the
+ *    matching *_workspace_size call.
+ *  - Device calls are asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Launch failures come back as PA_ERR_CUDA;
+ *    argument checks are done on the host before anything is enqueued, so an
+ *    error return means nothing was launched.
+ *  - Pool calls are host-only, single-threaded per pool, and never touch KV
+ *    bytes.
+ *
+ * Data layout in device memory
+ *  - K pool: [num_blocks][num_kv_heads][block_size][head_dim].
+ *  - V pool: the same for PA_F32 / PA_BF16 caches; d-major
+ *    [num_blocks][num_kv_heads][head_dim][block_size] for PA_FP8_E4M3 caches.
+ *  - Flat slot of the token at position p of a sequence with block table T:
+ *    T[p / block_size] * block_size + p % block_size.
+ *  - Queries, new K/V rows and outputs are row-major [rows][heads][head_dim]
+ *    in the query dtype.  Query head h reads KV head h / (num_q_heads /
+ *    num_kv_heads).
+ *  - Block tables: int32 [num_seqs][max_blocks_per_seq], row s padded past
+ *    its last block with any value (never read).
+ *  - All base pointers 16-byte aligned.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or id */
+  PA_ERR_UNSUPPORTED = 2, /* valid but not built: dtype/head_dim/block_size/group combination */
+  PA_ERR_NO_BLOCKS = 3,   /* pool exhausted; the pool is left unchanged */
+  PA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  PA_ERR_STATE = 5        /* inconsistent pool state (e.g. ref_cnt underflow) */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
+
+/* Shape and storage of one layer's paged cache. */
+typedef struct {
+  int32_t num_blocks;   /* physical blocks in the pool */
+  int32_t block_size;   /* tokens per block: 16 or 32 */
+  int32_t num_kv_heads;
+  int32_t num_q_heads;  /* a multiple of num_kv_heads */
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t kv_dtype;     /* pa_dtype of the pool */
+  int32_t q_dtype;      /* pa_dtype of queries, new K/V and outputs: PA_F32 or PA_BF16 */
+  float k_scale;        /* per-tensor scales of an e4m3 pool (stored = e4m3(x / scale)); */
+  float v_scale;        /* ignored for fp32/bf16 pools */
+} pa_cache_desc;
+
+/* Message for the last failing call on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Library version string. */
+const char* pa_version(void);
+
+/* Bytes one physical block holds for K and V together:
+ * 2 * block_size * num_kv_heads * head_dim * sizeof(kv element)
+ * ("vLLM innenfra ...", paragraph 2).  Returns 0 for an invalid desc. */
+size_t pa_block_bytes(const pa_cache_desc* desc);
+
+/* ---- device calls --------------------------------------------------------- */
+
+/* pa_cache_write: scatter this step's new K and V rows into their blocks.
+ * Follows the "write(blocks[-1], kv)" step of the block-table snippet on "49
+ * vLLM / PagedAttention"; slot_mapping carries each new token's flat slot.
+ *   k_new, v_new   device, [num_tokens][num_kv_heads][head_dim], q_dtype
+ *   slot_mapping   device, int64 [num_tokens]; a negative slot is skipped, and
+ *                  so is a slot >= num_blocks * block_size
+ *   k_cache/v_cache device pools (layout above), written in place
+ * fp32 -> fp32 and bf16 -> bf16 are bit copies; fp32/bf16 -> e4m3 stores
+ * e4m3(fp32(x) / fp32(scale)) rounded to nearest-even with saturation to
+ * +-448.  bf16 -> fp32 and fp32 -> bf16 are PA_ERR_UNSUPPORTED.  Two new
+ * tokens with the same slot race (last writer unspecified). */
+int pa_cache_write(const pa_cache_desc* desc, const void* k_new, const void* v_new,
+                   const int64_t* slot_mapping, int32_t num_tokens, void* k_cache, void* v_cache,
+                   void* stream);
+
+/* Scratch bytes pa_decode needs for num_seqs sequences on the current device. */
+size_t pa_decode_workspace_size(const pa_cache_desc* desc, int32_t num_seqs);
+
+/* pa_decode: one decode step of paged attention.  Sequence s has one query
+ * row (row s of q) at position seq_lens[s] - 1 and attends its keys
+ * 0 .. seq_lens[s] - 1, gathered through block_tables[s]; seq_lens counts
+ * the token written this step.  out[s][h][:] = softmax(scale * q K^T) V.
+ *   q           device, [num_seqs][num_q_heads][head_dim], q_dtype
+ *   block_tables device, int32 [num_seqs][max_blocks_per_seq]
+ *   seq_lens    device, int32 [num_seqs]; 0 gives a zero output row
+ *   out         device, [num_seqs][num_q_heads][head_dim], q_dtype
+ *   workspace   device, >= pa_decode_workspace_size bytes, 256-byte aligned.
+ *               Its first 4 bytes are an error word the kernels set (never
+ *               clear) if a bounded internal wait times out; zero it once to
+ *               arm it and read it after the stream synchronises.  The rest
+ *               needs no initialisation.  Calls sharing a workspace must not
+ *               overlap on the GPU.
+ * Long contexts are split over many CTAs (split-K over blocks) and merged
+ * with a log-sum-exp combine; the split points depend only on seq_lens and
+ * the device, so a result does not depend on where the blocks sit. */
+int pa_decode(const pa_cache_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+              int32_t num_seqs, float scale, void* out, void* workspace, size_t workspace_bytes,
+              void* stream);
+
+/* Scratch bytes pa_decode_chunked_prefill needs. */
+size_t pa_prefill_workspace_size(const pa_cache_desc* desc, int32_t num_seqs, int32_t num_tokens);
+
+/* pa_decode_chunked_prefill: one mixed step where some sequences add a chunk
+ * of prompt tokens and others decode one token ("vLLM innenfra ...", the
+ * step() list, item 1, and the paragraph on continuous batching: prefill and
+ * decode share a step).  Sequence s owns query rows
+ * query_start_loc[s] .. query_start_loc[s+1]-1 (q_len_s rows); its row i sits
+ * at position seq_lens[s] - q_len_s + i and attends keys 0 .. that position
+ * (causal).  seq_lens counts every token including this step's.  The new
+ * tokens' K/V must already be in the pool (pa_cache_write).
+ *   q, out          device, [num_tokens][num_q_heads][head_dim], q_dtype
+ *   query_start_loc device, int32 [num_seqs + 1], query_start_loc[0] = 0,
+ *                   non-decreasing, query_start_loc[num_seqs] = num_tokens
+ *   seq_lens        device, int32 [num_seqs], seq_lens[s] >= q_len_s
+ *   max_q_len       host, >= every q_len_s
+ *   workspace       as for pa_decode, sized by pa_prefill_workspace_size. */
+int pa_decode_chunked_prefill(const pa_cache_desc* desc, const void* q, const void* k_cache,
+                              const void* v_cache, const int32_t* block_tables,
+                              int32_t max_blocks_per_seq, const int32_t* query_start_loc,
+                              const int32_t* seq_lens, int32_t num_seqs, int32_t num_tokens,
+                              int32_t max_q_len, float scale, void* out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* ---- host block pool --------------------------------------------------------
+ * The block manager of "PagedAttention：KV cache 即虚拟内存（block manager &
+ * 碎片）", section 深入原理: free_block_queue is a doubly linked list in
+ * eviction order (pop head to allocate, push tail to release, both O(1));
+ * every block has a ref_cnt; full blocks are keyed by a hash of their tokens
+ * and their parent's hash so that equal prefixes share blocks (touch()
+ * raises ref_cnt); a finished sequence decrements ref_cnt and releases a
+ * block at 0.  Decoding takes a new block exactly when the token being
+ * appended starts one (block-table snippet on "49 vLLM / PagedAttention").
+ *
+ * Details the pages leave open, as implemented:
+ *  - block hash: FNV-1a 64 over the parent hash (8 bytes little endian, 0
+ *    for the first block) then the block's token ids (int32 little endian);
+ *    a hit also compares the stored token ids;
+ *  - sharing covers the longest run of leading full blocks found in the
+ *    map; a newly allocated full block enters the map unless its hash is
+ *    already there;
+ *  - a released block keeps its hash while parked in the free queue and can
+ *    still be shared (touch() unlinks it); popping it for reuse evicts it;
+ *  - release walks a sequence's blocks in reverse logical order;
+ *  - every allocation is all-or-nothing (PA_ERR_NO_BLOCKS changes nothing);
+ *  - blocks filled by pa_pool_append are never hashed. */
+
+typedef struct pa_pool pa_pool;
+
+/* initial_free_order: NULL for 0..num_blocks-1, else a permutation of it
+ * (head first).  *out receives a handle owned by the library. */
+int pa_pool_create(int32_t num_blocks, int32_t block_size, const int32_t* initial_free_order,
+                   pa_pool** out);
+void pa_pool_destroy(pa_pool* pool);
+
+/* Admit a prompt of num_tokens (token_ids NULL: no prefix sharing).
+ * num_cached_tokens (nullable) receives the tokens covered by shared blocks. */
+int pa_pool_add_seq(pa_pool* pool, int64_t seq_id, const int32_t* token_ids, int32_t num_tokens,
+                    int32_t* num_cached_tokens);
+
+/* Grow a sequence by n_new tokens; slots_out[n_new] receives their flat slots. */
+int pa_pool_append(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slots_out);
+
+/* Flat slots of positions [start, start + n) of a sequence (all < its length). */
+int pa_pool_slots(const pa_pool* pool, int64_t seq_id, int32_t start, int32_t n, int64_t* slots_out);
+
+/* Release a sequence: ref_cnt-- per block, blocks reaching 0 go to the tail. */
+int pa_pool_free_seq(pa_pool* pool, int64_t seq_id);
+
+/* Copy a sequence's block table into out[cap]; *n receives its length
+ * (PA_ERR_INVALID_ARG if cap is too small; *n is still set). */
+int pa_pool_block_table(const pa_pool* pool, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n);
+
+/* Fill out[num_seqs][max_blocks] with the tables of seq_ids, padding with -1. */
+int pa_pool_block_tables(const pa_pool* pool, const int64_t* seq_ids, int32_t num_seqs,
+                         int32_t max_blocks, int32_t* out);
+
+/* Tokens a sequence holds. */
+int pa_pool_num_tokens(const pa_pool* pool, int64_t seq_id, int32_t* n);
+
+/* ref_cnt of a block (-1 if out of range). */
+int32_t pa_pool_ref_cnt(const pa_pool* pool, int32_t block);
+
+/* Blocks in the free queue. */
+int32_t pa_pool_num_free(const pa_pool* pool);
+
+/* The free queue head to tail into out[cap]; *n receives its length. */
+int pa_pool_free_order(const pa_pool* pool, int32_t* out, int32_t cap, int32_t* n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -73,6 +73,7 @@ class Workload:
     k_scale: float = 1.0
     v_scale: float = 1.0
     _fixed: Optional[dict] = field(default=None, repr=False)
+    _amax: Optional[dict] = field(default=None, repr=False)
 
     # ---- shape helpers (no method arithmetic) --------------------------------
     @property
@@ -119,9 +120,15 @@ class Workload:
         return k, v
 
     def prior_kv(self, s: int):
-        """K, V of sequence s's cached context in the input dtype (torch, CPU)."""
+        """K, V of sequence s's cached context in the input dtype (torch, CPU).
+        Records the draws' absolute maxima for fp8_scales_from_draws."""
         k, v = self.prior_kv_f32(s)
-        return _cast(k, self.q_dtype), _cast(v, self.q_dtype)
+        k, v = _cast(k, self.q_dtype), _cast(v, self.q_dtype)
+        if self._amax is None:
+            self._amax = {}
+        self._amax[s] = (float(k.abs().max()) if k.numel() else 0.0,
+                         float(v.abs().max()) if v.numel() else 0.0)
+        return k, v
 
     def new_kv(self):
         """K, V of this step's new tokens: [num_new_tokens][kv_heads][head_dim]."""
@@ -149,10 +156,10 @@ class Workload:
         the input dtype; sets and returns (k_scale, v_scale)."""
         ak = av = 0.0
         for s in range(self.num_seqs):
-            k, v = self.prior_kv(s)
-            if k.numel():
-                ak = max(ak, float(k.abs().max()))
-                av = max(av, float(v.abs().max()))
+            if self._amax is None or s not in self._amax:
+                self.prior_kv(s)
+            ak = max(ak, self._amax[s][0])
+            av = max(av, self._amax[s][1])
         k, v = self.new_kv()
         if k.numel():
             ak = max(ak, float(k.abs().max()))

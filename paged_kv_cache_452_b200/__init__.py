@@ -1,0 +1,232 @@
+"""Paged KV-cache decode attention for B200 (sm_100a): a thin Python binding
+over the C ABI of libpa.so (include/pa.h).
+
+Every function here only marshals arguments (torch tensors -> device
+pointers, the current CUDA stream) and calls the library function of the
+same name; all work runs in the library's CUDA kernels or its C++ block pool.
+Importing fails loudly if libpa.so has not been built
+(``python -m paged_kv_cache_452_b200.build``); there is no fallback.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+from ._lib import LIB_PATH, PaError, lib  # noqa: F401
+
+PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+_CODES = {"f32": PA_F32, "bf16": PA_BF16, "e4m3": PA_FP8_E4M3}
+_TORCH = {PA_F32: torch.float32, PA_BF16: torch.bfloat16, PA_FP8_E4M3: torch.uint8}
+_NAMES = {v: k for k, v in _CODES.items()}
+
+
+class CacheDesc(ctypes.Structure):
+    """pa_cache_desc: shape and storage of one layer's paged cache."""
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("q_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float)]
+
+    @classmethod
+    def make(cls, num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, kv_dtype="bf16",
+             q_dtype="bf16", k_scale=1.0, v_scale=1.0):
+        kv = _CODES.get(kv_dtype, kv_dtype)
+        q = _CODES.get(q_dtype, q_dtype)
+        return cls(num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, kv, q,
+                   float(k_scale), float(v_scale))
+
+    @property
+    def group(self):
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def kv_torch_dtype(self):
+        return _TORCH[self.kv_dtype]
+
+    @property
+    def q_torch_dtype(self):
+        return _TORCH[self.q_dtype]
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise PaError(rc, f"{what}: {lib().pa_last_error().decode()}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def pa_block_bytes(desc: CacheDesc) -> int:
+    return int(lib().pa_block_bytes(ctypes.byref(desc)))
+
+
+def alloc_cache(desc: CacheDesc, device, fill=None):
+    """Allocate (K pool, V pool) as torch tensors in the library's layout:
+    K [NB][Hkv][bs][D]; V the same, or [NB][Hkv][D][bs] for an e4m3 pool.
+    fill: optional element value (a raw byte for e4m3)."""
+    nb, bs, h, d = desc.num_blocks, desc.block_size, desc.num_kv_heads, desc.head_dim
+    dt = desc.kv_torch_dtype
+    k = torch.empty((nb, h, bs, d), dtype=dt, device=device)
+    v = torch.empty((nb, h, d, bs) if desc.kv_dtype == PA_FP8_E4M3 else (nb, h, bs, d), dtype=dt,
+                    device=device)
+    if fill is not None:
+        k.fill_(fill)
+        v.fill_(fill)
+    return k, v
+
+
+def pa_cache_write(desc, k_new, v_new, slot_mapping, k_cache, v_cache, stream=None):
+    """Scatter new K/V rows [T][Hkv][D] into the pools through int64 slots."""
+    n = int(slot_mapping.shape[0])
+    _check(lib().pa_cache_write(ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), n,
+                                _ptr(k_cache), _ptr(v_cache), _stream(stream)), "pa_cache_write")
+
+
+def pa_decode_workspace_size(desc, num_seqs) -> int:
+    n = int(lib().pa_decode_workspace_size(ctypes.byref(desc), int(num_seqs)))
+    if n == 0:
+        raise PaError(1, "pa_decode_workspace_size: " + lib().pa_last_error().decode())
+    return n
+
+
+def pa_prefill_workspace_size(desc, num_seqs, num_tokens) -> int:
+    n = int(lib().pa_prefill_workspace_size(ctypes.byref(desc), int(num_seqs), int(num_tokens)))
+    if n == 0:
+        raise PaError(1, "pa_prefill_workspace_size: " + lib().pa_last_error().decode())
+    return n
+
+
+def alloc_workspace(nbytes, device):
+    """Caller-owned scratch; the error word in its first bytes starts at zero."""
+    return torch.zeros(int(nbytes), dtype=torch.uint8, device=device)
+
+
+def workspace_error(workspace) -> int:
+    """The error word a kernel sets when a bounded wait times out (1) or a
+    block table entry is outside the pool (2).  Synchronises."""
+    return int(workspace[:4].view(torch.int32).item())
+
+
+def pa_decode(desc, q, k_cache, v_cache, block_tables, seq_lens, scale, out, workspace, stream=None):
+    """One decode step: q [S][Hq][D] attends seq_lens[s] keys via block_tables [S][max_blocks]."""
+    s = int(seq_lens.shape[0])
+    _check(lib().pa_decode(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                           int(block_tables.shape[1]), _ptr(seq_lens), s, float(scale), _ptr(out),
+                           _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                           _stream(stream)), "pa_decode")
+
+
+def pa_decode_chunked_prefill(desc, q, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
+                              max_q_len, scale, out, workspace, stream=None):
+    """A mixed step: sequence s owns rows query_start_loc[s]..query_start_loc[s+1]-1 (causal)."""
+    s = int(seq_lens.shape[0])
+    _check(lib().pa_decode_chunked_prefill(
+        ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        int(block_tables.shape[1]), _ptr(query_start_loc), _ptr(seq_lens), s, int(q.shape[0]),
+        int(max_q_len), float(scale), _ptr(out), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _stream(stream)),
+        "pa_decode_chunked_prefill")
+
+
+def default_scale(head_dim):
+    return 1.0 / math.sqrt(head_dim)
+
+
+class BlockPool:
+    """Host block pool (pa_pool_*): free_block_queue, ref_cnt, prefix sharing."""
+
+    def __init__(self, num_blocks, block_size, initial_free_order=None):
+        self._lib = lib()
+        h = ctypes.c_void_p()
+        arr = None
+        if initial_free_order is not None:
+            order = [int(b) for b in initial_free_order]
+            if len(order) != num_blocks:
+                raise PaError(1, "initial_free_order must have num_blocks entries")
+            arr = (ctypes.c_int32 * num_blocks)(*order)
+        _check(self._lib.pa_pool_create(int(num_blocks), int(block_size), arr, ctypes.byref(h)),
+               "pa_pool_create")
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if self._h:
+            self._lib.pa_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id, num_tokens, token_ids=None) -> int:
+        arr = None
+        if token_ids is not None:
+            ids = [int(t) for t in token_ids]
+            arr = (ctypes.c_int32 * len(ids))(*ids)
+        cached = ctypes.c_int32(0)
+        _check(self._lib.pa_pool_add_seq(self._h, int(seq_id), arr, int(num_tokens), ctypes.byref(cached)),
+               "pa_pool_add_seq")
+        return cached.value
+
+    def append(self, seq_id, n_new):
+        out = (ctypes.c_int64 * max(1, n_new))()
+        _check(self._lib.pa_pool_append(self._h, int(seq_id), int(n_new), out), "pa_pool_append")
+        return list(out[:n_new])
+
+    def slots(self, seq_id, start, n):
+        out = (ctypes.c_int64 * max(1, n))()
+        _check(self._lib.pa_pool_slots(self._h, int(seq_id), int(start), int(n), out), "pa_pool_slots")
+        return list(out[:n])
+
+    def free_seq(self, seq_id):
+        _check(self._lib.pa_pool_free_seq(self._h, int(seq_id)), "pa_pool_free_seq")
+
+    def num_tokens(self, seq_id):
+        n = ctypes.c_int32()
+        _check(self._lib.pa_pool_num_tokens(self._h, int(seq_id), ctypes.byref(n)), "pa_pool_num_tokens")
+        return n.value
+
+    def block_table(self, seq_id):
+        n = ctypes.c_int32()
+        self._lib.pa_pool_block_table(self._h, int(seq_id), None, 0, ctypes.byref(n))
+        out = (ctypes.c_int32 * max(1, n.value))()
+        _check(self._lib.pa_pool_block_table(self._h, int(seq_id), out, n.value, ctypes.byref(n)),
+               "pa_pool_block_table")
+        return list(out[:n.value])
+
+    def block_tables(self, seq_ids, max_blocks):
+        """Padded int32 table [len(seq_ids)][max_blocks] as a CPU torch tensor."""
+        ids = (ctypes.c_int64 * max(1, len(seq_ids)))(*[int(s) for s in seq_ids])
+        out = torch.empty((len(seq_ids), max_blocks), dtype=torch.int32)
+        _check(self._lib.pa_pool_block_tables(self._h, ids, len(seq_ids), int(max_blocks),
+                                              ctypes.c_void_p(out.data_ptr())), "pa_pool_block_tables")
+        return out
+
+    def ref_cnt(self, block):
+        return int(self._lib.pa_pool_ref_cnt(self._h, int(block)))
+
+    def num_free(self):
+        return int(self._lib.pa_pool_num_free(self._h))
+
+    def free_order(self):
+        n = ctypes.c_int32()
+        cap = self.num_blocks
+        out = (ctypes.c_int32 * max(1, cap))()
+        _check(self._lib.pa_pool_free_order(self._h, out, cap, ctypes.byref(n)), "pa_pool_free_order")
+        return list(out[:n.value])

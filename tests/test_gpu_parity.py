@@ -1,0 +1,196 @@
+"""CUDA path against the CPU oracle, through the C ABI.
+
+Bit-exact: block tables and slot mappings (C++ pool vs pool model) and every
+cache element written this step or at set-up (pa_cache_write vs the oracle's
+write, e4m3 quantisation included).  Attention: max abs error against the
+fp64 oracle within 1e-4 (fp32), 2e-2 (bf16), 6e-2 (e4m3, against the oracle
+on the dequantised values).
+"""
+import numpy as np
+import pytest
+import torch
+
+import pa_workloads as W
+import paged_kv_cache_452_b200 as pa
+from oracle.workload import expected
+from paged_kv_cache_452_b200 import runner
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2, "e4m3": 6e-2}
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t.view(torch.int32).numpy()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy()
+    return t.numpy()
+
+
+def check_cache(wl, b, exp):
+    """Every position of every checked sequence: GPU pool bytes == oracle pool bytes."""
+    bs = wl.block_size
+    kc, vc = exp["k_cache"], exp["v_cache"]
+    for s in exp["seqs"]:
+        n = int(wl.context_lens[s] + wl.q_lens[s])
+        if n == 0:
+            continue
+        pos = np.arange(n)
+        blk = exp["tables"][s, pos // bs]
+        cblk = exp["compact_tables"][s, pos // bs]
+        off = pos % bs
+        bi = torch.from_numpy(blk.astype(np.int64)).to(b.k_cache.device)
+        oi = torch.from_numpy(off.astype(np.int64)).to(b.k_cache.device)
+        gk = bits(b.k_cache[bi, :, oi, :])
+        ok_ = kc[cblk, :, off, :]
+        if wl.kv_dtype == "e4m3":
+            gv = bits(b.v_cache[bi, :, :, oi])
+            ov = vc[cblk, :, :, off]
+        else:
+            gv = bits(b.v_cache[bi, :, oi, :])
+            ov = vc[cblk, :, off, :]
+        assert np.array_equal(gk.view(ok_.dtype), ok_), f"K bytes differ in sequence {s}"
+        assert np.array_equal(gv.view(ov.dtype), ov), f"V bytes differ in sequence {s}"
+
+
+def run_and_check(wl, device, seqs=None):
+    b = runner.setup(wl, device)
+    runner.step(b)
+    torch.cuda.synchronize()
+    exp = expected(wl, seqs)
+    assert np.array_equal(b.tables_host.numpy(), exp["tables"])
+    assert np.array_equal(b.slots_host.numpy(), exp["step_slots"])
+    assert b.num_cached == exp["num_cached"]
+    check_cache(wl, b, exp)
+    out = b.out.detach().cpu().to(torch.float64).numpy()[exp["rows"]]
+    assert np.isfinite(out).all()
+    err = float(np.abs(out - exp["out"]).max()) if out.size else 0.0
+    assert err <= TOL[wl.kv_dtype], f"{wl.name}: max abs error {err}"
+    assert pa.workspace_error(b.workspace) == 0
+    return b, err
+
+
+SMALL = ["tiny_fp32", "gqa_bf16", "prefix_bf16", "fp8_long", "mixed_prefill_bs16", "mixed_prefill_bs32"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_workload_small(name, cuda_device):
+    run_and_check(W.make(name, "small"), cuda_device)
+
+
+EDGE = {
+    # empty context (attends only the new token), block boundaries, ragged tails
+    "bounds_bs16": dict(context_lens=[0, 1, 15, 16, 17, 31, 32, 33, 47, 48]),
+    "bounds_bs32": dict(context_lens=[0, 1, 31, 32, 33, 63, 64, 65], block_size=32),
+    "bounds_fp8_bs16": dict(context_lens=[0, 15, 16, 17, 100], kv_dtype="e4m3"),
+    "bounds_fp8_bs32": dict(context_lens=[0, 31, 32, 33, 200], kv_dtype="e4m3", block_size=32),
+    "group2": dict(context_lens=[5, 80, 300], num_q_heads=4, num_kv_heads=2),
+    "group8": dict(context_lens=[5, 80, 300], num_q_heads=16, num_kv_heads=2),
+    "group8_fp8": dict(context_lens=[5, 80, 300], num_q_heads=16, num_kv_heads=2, kv_dtype="e4m3"),
+    "head64": dict(context_lens=[3, 64, 129], head_dim=64),
+    "head64_bs32": dict(context_lens=[3, 64, 129], head_dim=64, block_size=32),
+    "mha_bf16": dict(context_lens=[7, 100], num_q_heads=4, num_kv_heads=4),  # group 1: CUDA cores
+    "group16_bf16": dict(context_lens=[7, 100], num_q_heads=32, num_kv_heads=2),  # group > 8: CUDA cores
+    "fp32_gqa": dict(context_lens=[9, 70], kv_dtype="f32", q_dtype="f32", num_q_heads=8, num_kv_heads=2),
+    "fp8_f32_queries": dict(context_lens=[9, 70], kv_dtype="e4m3", q_dtype="f32"),
+    "one_long": dict(context_lens=[5000], num_q_heads=8, num_kv_heads=8 // 4),  # split over many CTAs
+    "many_short": dict(context_lens=list(range(0, 700, 1)), num_q_heads=4, num_kv_heads=2, head_dim=64),
+    "single": dict(context_lens=[1]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(EDGE))
+def test_edge_cases(case, cuda_device):
+    run_and_check(W.custom(case, **EDGE[case]), cuda_device)
+
+
+def test_mixed_edge_cases(cuda_device):
+    # prefill chunks with no prior context, a 1-token chunk, chunks crossing blocks
+    wl = W.custom("mixed_edges", context_lens=[0, 0, 17, 40, 3, 100], q_lens=[1, 20, 33, 1, 16, 1])
+    run_and_check(wl, cuda_device)
+
+
+def test_paged_output_equals_contiguous_output(cuda_device):
+    """Paging changes nothing: the same draws through a shuffled free list and
+    through an identity free list (contiguous blocks) give bit-identical
+    outputs, because split points depend only on the lengths."""
+    a = W.gqa_bf16("small")
+    b = W.gqa_bf16("small")
+    b.free_order = np.arange(b.num_blocks, dtype=np.int32)
+    ra = runner.setup(a, cuda_device)
+    rb = runner.setup(b, cuda_device)
+    runner.step(ra)
+    runner.step(rb)
+    torch.cuda.synchronize()
+    assert not torch.equal(ra.tables, rb.tables)
+    assert torch.equal(ra.out.view(torch.int16), rb.out.view(torch.int16))
+
+
+def test_prefix_sharing_leaves_output_unchanged(cuda_device):
+    """Sequences that share prefix blocks give the same bits as with private
+    copies of the prefix (the pages: KV byte-identical, output unchanged)."""
+    a = W.prefix_bf16("small")
+    b = W.prefix_bf16("small")
+    b.sharing = None  # no token ids: every sequence gets private blocks
+    b.prefix_len = a.prefix_len
+
+    # same values: b draws its prefix from the shared stream too
+    def prior_kv_f32(s, _a=a):
+        return _a.prior_kv_f32(s)
+    b.prior_kv_f32 = prior_kv_f32
+    b.num_blocks = a.num_blocks + a.prefix_len // a.block_size * int(a.sharing.sum())
+    b.free_order = np.arange(b.num_blocks, dtype=np.int32)
+    ra = runner.setup(a, cuda_device)
+    rb = runner.setup(b, cuda_device)
+    runner.step(ra)
+    runner.step(rb)
+    torch.cuda.synchronize()
+    shared = ra.tables[0, : a.prefix_len // a.block_size]
+    assert torch.equal(ra.tables[1, : a.prefix_len // a.block_size], shared)
+    assert not torch.equal(rb.tables[1, : a.prefix_len // a.block_size], rb.tables[0, : a.prefix_len // a.block_size])
+    assert torch.equal(ra.out.view(torch.int16), rb.out.view(torch.int16))
+
+
+def test_repeated_steps_are_deterministic(cuda_device):
+    wl = W.fp8_long("small")
+    b = runner.setup(wl, cuda_device)
+    runner.step(b)
+    first = b.out.clone()
+    for _ in range(3):
+        runner.attend(b)
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int16), b.out.view(torch.int16))
+
+
+def test_bad_table_entry_is_flagged_not_faulted(cuda_device):
+    wl = W.gqa_bf16("small")
+    b = runner.setup(wl, cuda_device)
+    runner.step(b)
+    b.tables[0, 0] = wl.num_blocks + 5  # past the pool: the kernel flags it and reads block 0
+    runner.attend(b)
+    torch.cuda.synchronize()
+    assert pa.workspace_error(b.workspace) == 2
+
+
+def test_context_longer_than_table_row_is_flagged(cuda_device):
+    wl = W.gqa_bf16("small")
+    b = runner.setup(wl, cuda_device)
+    runner.step(b)
+    b.seq_lens[0] = b.tables.shape[1] * wl.block_size + 40  # beyond the row: flagged and clamped
+    runner.attend(b)
+    torch.cuda.synchronize()
+    assert pa.workspace_error(b.workspace) == 3
+
+
+FULL = [("gqa_bf16", [0, 17, 63]), ("prefix_bf16", [0, 1, 127, 128, 255]), ("fp8_long", [0, 77]),
+        ("mixed_prefill_bs16", [0, 7, 8, 255]), ("mixed_prefill_bs32", [3, 100])]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,seqs", FULL)
+def test_workload_full_size_sampled(name, seqs, cuda_device):
+    """Full-size workload, launched exactly as bench.py does; the oracle checks
+    sampled sequences (their rows, their cache bytes) and the full tables."""
+    run_and_check(W.make(name, "full"), cuda_device, seqs)

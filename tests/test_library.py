@@ -1,0 +1,80 @@
+"""Host-side checks of the C ABI library (no GPU needed): every declared
+symbol is exported, the byte accounting matches the pages' formula, and bad
+arguments are rejected before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_452_b200 as pa
+from oracle import admission
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "pa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = declared_functions()
+    assert len(names) >= 20
+    L = ctypes.CDLL(pa.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    from paged_kv_cache_452_b200._lib import SIGNATURES
+    assert set(SIGNATURES) == set(names)
+
+
+def test_version_and_error_string():
+    assert b"sm_100a" in pa.lib().pa_version()
+    assert pa.lib().pa_last_error() == b""
+
+
+@pytest.mark.parametrize("bs,hkv,d,kv,eb", [(16, 8, 128, "bf16", 2), (16, 8, 128, "e4m3", 1),
+                                             (32, 8, 128, "bf16", 2), (16, 2, 64, "f32", 4)])
+def test_block_bytes_matches_formula(bs, hkv, d, kv, eb):
+    desc = pa.CacheDesc.make(100, bs, hkv, hkv * 4, d, kv, "bf16" if kv != "f32" else "f32", 0.5, 0.5)
+    assert pa.pa_block_bytes(desc) == admission.block_bytes(bs, hkv, d, eb)
+
+
+def _call_write(desc, n=1, ptr=16):
+    slots = ctypes.c_void_p(ptr)
+    return pa.lib().pa_cache_write(ctypes.byref(desc) if desc is not None else None, ptr, ptr, slots, n,
+                                   ptr, ptr, None)
+
+
+def test_cache_write_rejects_bad_arguments_on_host():
+    good = pa.CacheDesc.make(16, 16, 2, 4, 64, "bf16", "bf16")
+    assert _call_write(None) == 1
+    assert b"desc is NULL" in pa.lib().pa_last_error()
+    assert _call_write(good, n=0) == 0  # nothing to do, nothing launched
+    assert _call_write(good, n=-1) == 1
+    assert _call_write(good, ptr=18) == 1  # misaligned
+    bad_bs = pa.CacheDesc.make(16, 8, 2, 4, 64, "bf16", "bf16")
+    assert _call_write(bad_bs) == 2  # block size 8 not built
+    bad_d = pa.CacheDesc.make(16, 16, 2, 4, 96, "bf16", "bf16")
+    assert _call_write(bad_d) == 2
+    bad_g = pa.CacheDesc.make(16, 16, 3, 4, 64, "bf16", "bf16")
+    assert _call_write(bad_g) == 1  # 4 query heads over 3 KV heads
+    mixed = pa.CacheDesc.make(16, 16, 2, 4, 64, "f32", "bf16")
+    assert _call_write(mixed) == 2  # bf16 rows into an fp32 pool
+    no_scale = pa.CacheDesc.make(16, 16, 2, 4, 128, "e4m3", "bf16", 0.0, 1.0)
+    assert _call_write(no_scale) == 1
+
+
+def test_decode_rejects_bad_arguments_on_host():
+    desc = pa.CacheDesc.make(16, 16, 2, 8, 128, "bf16", "bf16")
+    L = pa.lib()
+    p = 256
+    rc = L.pa_decode(ctypes.byref(desc), p, p, p, p, 4, p, -1, 1.0, p, p, 1 << 20, None)
+    assert rc == 1
+    rc = L.pa_decode(ctypes.byref(desc), p, p, p, p, 4, p, 0, 1.0, p, p, 1 << 20, None)
+    assert rc == 0  # empty batch
+    rc = L.pa_decode(ctypes.byref(desc), p, p, p, p, 4, p, 3, 1.0, p, p + 16, 1 << 20, None)
+    assert rc == 1 and b"misaligned" in L.pa_last_error()
+    rc = L.pa_decode(ctypes.byref(desc), None, p, p, p, 4, p, 3, 1.0, p, p, 1 << 20, None)
+    assert rc == 1
