@@ -196,6 +196,16 @@ def bench_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _time(fn, steps, stream):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def bench_ours(args):
     world, rank, local = dist_setup(args)
     if not torch.cuda.is_available():
@@ -212,38 +222,40 @@ def bench_ours(args):
     alg_bytes, kv_bytes = algorithmic_bytes(wl)
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        runner.step(batches[i & 1])
-
+    # eager warm-up through the public API, then one CUDA graph per pool copy
+    # for the step (cache write + decode) and for the decode alone, as a
+    # serving loop would replay them
     for i in range(args.warmup):
-        step(i)
+        runner.step(batches[i & 1])
+    torch.cuda.synchronize()
+    g_step, g_attend = [], []
+    for b in batches:
+        gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gs):
+            runner.step(b)
+        with torch.cuda.graph(ga):
+            runner.attend(b)
+        g_step.append(gs)
+        g_attend.append(ga)
+    for i in range(args.warmup):
+        g_step[i & 1].replay()
+        g_attend[i & 1].replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local) if rank == 0 else None
     time.sleep(0.2 if sampler else 0)
     barrier(world)
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    ev1.record(stream)
+    ms = _time(lambda i: g_step[i & 1].replay(), args.steps, stream)
     torch.cuda.synchronize()
     barrier(world)
-    ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, device)
-
-    # the dominant call, pa_decode (decode kernel + its log-sum-exp combine),
-    # timed per launch with events on its stream over the same number of steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        runner.write_step(batches[i & 1])
-        evs[i][0].record(stream)
-        runner.attend(batches[i & 1])
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
+    ms = reduce_max(ms, world, device)
+    # the dominant kernel, pa_decode's single launch, per launch: replays of a
+    # graph holding only it, events on the replay stream
+    attend_ms = reduce_max(_time(lambda i: g_attend[i & 1].replay(), args.steps, stream), world, device)
     clocks = sampler.stop() if sampler else None
-    attend_ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world, device)
+    # the same step issued launch by launch from Python (no graph)
+    eager_ms = reduce_max(_time(lambda i: runner.step(batches[i & 1]), args.steps, stream), world, device)
 
     # end to end through the public API with host buffers: H2D of the step's
     # inputs from pinned memory, write + decode, D2H of the output
@@ -252,27 +264,24 @@ def bench_ours(args):
     out_host = torch.empty(b0.out.shape, dtype=b0.out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
-    for i in range(max(1, args.warmup)):
+
+    def e2e_step(i):
         for k, t in host.items():
             getattr(b0, k).copy_(t, non_blocking=True)
         runner.step(b0)
         out_host.copy_(b0.out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        for k, t in host.items():
-            getattr(b0, k).copy_(t, non_blocking=True)
-        runner.step(b0)
-        out_host.copy_(b0.out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, device)
+    e2e_ms = reduce_max(_time(e2e_step, args.steps, stream), world, device)
 
     errs = [pa.workspace_error(b.workspace) for b in batches]
     if any(errs):
         raise SystemExit(f"kernel error word set: {errs}")
+    for gg in g_step + g_attend:
+        del gg
 
     if rank != 0:
         if world > 1:
@@ -290,15 +299,17 @@ def bench_ours(args):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": wl.block_size,
                    "context_tokens": int((wl.context_lens + wl.q_lens).sum()), "kv_bytes": kv_bytes,
                    "algorithmic_bytes": alg_bytes, "parallelism": f"replicas x{world}",
+                   "step": "pa_cache_write + pa_decode, replayed as a CUDA graph",
                    "l2": "2 pool copies used alternately, each larger than L2"},
         "decode_tokens_per_s": world * wl.num_seqs / (ms * 1e-3),
-        "fraction_of_8tbs": world * alg_bytes / (ms * 1e-3) / 1e9 / 8000.0 / world,
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_tc_kernel + decode_combine_kernel)",
+        "fraction_of_8tbs": alg_bytes / (ms * 1e-3) / 1e9 / 8000.0,
+        "eager_ms_per_step": eager_ms,
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (pa_decode)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src, "traffic": None, "pa_decode_ms": attend_ms},
+                     "peak_source": src, "traffic": None, "kernel_ms": attend_ms},
         "e2e": {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:
@@ -311,7 +322,7 @@ def bench_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

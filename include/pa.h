@@ -111,11 +111,15 @@ size_t pa_decode_workspace_size(const pa_cache_desc* desc, int32_t num_seqs);
  *   block_tables device, int32 [num_seqs][max_blocks_per_seq]
  *   seq_lens    device, int32 [num_seqs]; 0 gives a zero output row
  *   out         device, [num_seqs][num_q_heads][head_dim], q_dtype
- *   workspace   device, >= pa_decode_workspace_size bytes, 256-byte aligned.
+ *   workspace   device, >= pa_decode_workspace_size bytes, 256-byte aligned,
+ *               zero-filled once before its first use; every call leaves it
+ *               ready for the next (also when replayed from a CUDA graph).
  *               Its first 4 bytes are an error word the kernels set (never
- *               clear) if a bounded internal wait times out; zero it once to
- *               arm it and read it after the stream synchronises.  The rest
- *               needs no initialisation.  Calls sharing a workspace must not
+ *               clear): 1 = a bounded internal wait timed out, 2 = a block
+ *               table entry outside [0, num_blocks) (read as block 0),
+ *               3 = a sequence longer than its table row (clamped).  Read it
+ *               after the stream synchronises; after any error, zero the
+ *               whole workspace again.  Calls sharing a workspace must not
  *               overlap on the GPU.
  * Long contexts are split over many CTAs (split-K over blocks) and merged
  * with a log-sum-exp combine; the split points depend only on seq_lens and

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -59,10 +60,13 @@ int check_desc(const pa_cache_desc* d, const char* who) {
 }
 
 int num_sms(int* out) {
+  static std::atomic<int> cached[64];  // per device, 0 = not yet queried
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess && dev < 64 && (*out = cached[dev].load(std::memory_order_relaxed)) > 0) return PA_OK;
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "cannot query the device: %s", cudaGetErrorString(e));
+  if (dev < 64) cached[dev].store(*out, std::memory_order_relaxed);
   return PA_OK;
 }
 
@@ -92,7 +96,41 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D map over a token-major pool viewed as rows of head_dim elements; one
 // box is [block_size rows][128 bytes] with 128-byte swizzle.
+int encode_kv_map(CUtensorMap* m, const void* base, int dt, const pa_cache_desc* d);
+
+// Encoded maps of recently used pools (a pool is normally reused every step):
+// a small table keyed by everything the encoding depends on.
 int make_kv_map(CUtensorMap* m, const void* base, int dt, const pa_cache_desc* d) {
+  struct Entry {
+    const void* base;
+    int dt, nb, hkv, bs, hd;
+    CUtensorMap map;
+  };
+  static Entry cache[16];
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const Entry& e = cache[i];
+      if (e.base == base && e.dt == dt && e.nb == d->num_blocks && e.hkv == d->num_kv_heads &&
+          e.bs == d->block_size && e.hd == d->head_dim) {
+        *m = e.map;
+        return PA_OK;
+      }
+    }
+  }
+  int rc = encode_kv_map(m, base, dt, d);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry& e = cache[next];
+  e = Entry{base, dt, d->num_blocks, d->num_kv_heads, d->block_size, d->head_dim, *m};
+  next = (next + 1) % 16;
+  if (used < 16) ++used;
+  return PA_OK;
+}
+
+int encode_kv_map(CUtensorMap* m, const void* base, int dt, const pa_cache_desc* d) {
   auto enc = encode_fn();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const int eb = elem_bytes(dt);
@@ -118,15 +156,15 @@ struct WsCarve {
   size_t bytes;
 };
 
-WsCarve carve(void* base, int num_seqs, int group, int head_dim, int sms) {
+WsCarve carve(void* base, int num_seqs, int num_kv_heads, int group, int head_dim, int sms) {
   WsCarve c;
   uint8_t* b = static_cast<uint8_t*>(base);
-  const size_t P = (size_t)decode_tc_grid(sms);
+  const size_t P = (size_t)decode_tc_workers(sms);
   size_t off = 0;
   c.ws.err = reinterpret_cast<int32_t*>(b + off);
   off += 256;
-  c.ws.prefix = reinterpret_cast<int32_t*>(b + off);
-  off += ((size_t)(num_seqs + 1) * 4 + 255) / 256 * 256;
+  c.ws.cnt = reinterpret_cast<unsigned int*>(b + off);
+  off += ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;
   c.ws.ml = reinterpret_cast<float*>(b + off);
   off += (2 * P * group * 2 * 4 + 255) / 256 * 256;
   c.ws.o = reinterpret_cast<float*>(b + off);
@@ -144,7 +182,7 @@ int run_decode_tc(const pa_cache_desc* d, const void* q, const void* k_cache, co
   int rc = num_sms(&sms);
   if (rc) return rc;
   const int group = d->num_q_heads / d->num_kv_heads;
-  WsCarve c = carve(workspace, num_seqs, group, d->head_dim, sms);
+  WsCarve c = carve(workspace, num_seqs, d->num_kv_heads, group, d->head_dim, sms);
   if (workspace_bytes < c.bytes)
     return fail(PA_ERR_INVALID_ARG, "%s: workspace %zu < %zu bytes", who, workspace_bytes, c.bytes);
   CUtensorMap tm_k, tm_v;
@@ -268,7 +306,7 @@ size_t pa_decode_workspace_size(const pa_cache_desc* d, int32_t num_seqs) {
   if (!use_tc(d)) return 256;
   int sms = 0;
   if (num_sms(&sms)) return 0;
-  return decode_tc_workspace_bytes(num_seqs, d->num_q_heads / d->num_kv_heads, d->head_dim, sms);
+  return decode_tc_workspace_bytes(num_seqs, d->num_kv_heads, d->num_q_heads / d->num_kv_heads, d->head_dim, sms);
 }
 
 static int check_attn_args(const pa_cache_desc* d, const void* q, const void* k_cache, const void* v_cache,
@@ -284,6 +322,9 @@ static int check_attn_args(const pa_cache_desc* d, const void* q, const void* k_
       !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 256))
     return fail(PA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
   if (num_seqs > 16384) return fail(PA_ERR_UNSUPPORTED, "%s: more than 16384 sequences per call", who);
+  // (sequence, kv head, block) tiles are indexed with 32-bit integers
+  if ((int64_t)num_seqs * max_blocks * d->num_kv_heads >= (int64_t)INT32_MAX)
+    return fail(PA_ERR_UNSUPPORTED, "%s: num_seqs * max_blocks_per_seq * num_kv_heads reaches 2^31", who);
   return PA_OK;
 }
 

@@ -9,26 +9,33 @@
 //
 // How, on sm_100a:
 //  * Work = (sequence, kv head, block) tiles.  The tiles of the whole batch
-//    are laid end to end and cut into one equal, contiguous range per CTA
-//    (persistent grid, 2 CTAs per SM), so a long context is split over
-//    several CTAs (split-K over blocks) and every SM streams the same number
-//    of bytes whatever the length mix.  A range cut inside a sequence leaves
-//    a partial (max, sum, unnormalised output) that a second kernel merges
-//    with a log-sum-exp combine; uncut sequences are finished in place.
-//  * One producer warp gathers tiles through the block table with TMA: the
-//    K tile (and the bf16 V tile) as 2-D tensor-map boxes of [block][128 B]
+//    are laid end to end and cut into one equal, contiguous range per warp
+//    (persistent grid, 2 CTAs of 4 warps per SM), so a long context is split
+//    over several warps (split-K over blocks) and every warp streams the
+//    same number of bytes whatever the length mix.  Each warp works alone:
+//    a (sequence, kv head) that lies wholly in its range is finished in
+//    registers and written out.  One cut by warp ranges is merged by the
+//    warp holding its first piece: that piece sits at the end of the warp's
+//    range, so it finishes after the later pieces, which sit at the starts
+//    of later warps' ranges.  Those store a partial (max, sum, unnormalised
+//    output) and count themselves in with a release reduction; the merging
+//    warp acquires the count (a bounded wait that normally ends at once) and
+//    folds the partials into its own state with a log-sum-exp combine in the
+//    MMA fragment layout.
+//  * Each warp gathers its tiles through the block table with TMA: the K
+//    tile (and the bf16 V tile) as 2-D tensor-map boxes of [block][128 B]
 //    with 128-byte swizzle, the e4m3 V tile (d-major, contiguous) as one bulk
-//    copy, into a ring of shared-memory stages guarded by mbarriers.  The
-//    query rows of each (sequence, kv head) come in by bulk copy too.
-//  * Four consumer warps take tiles round-robin.  GQA groups are packed with
+//    copy, into the warp's own ring of shared-memory stages, each guarded by
+//    an mbarrier.  A warp refills a stage as soon as it has consumed it, so
+//    every warp keeps its next tiles in flight and the load issue work is
+//    spread over all warps of the SM.
+//  * GQA groups are packed with
 //    keys on the MMA's M side and the group's query rows on N (8, padded):
 //    S^T = K Q^T and O^T += V^T P^T with mma.sync m16n8k16 (fp32 accumulate),
 //    an online softmax per query column, and P^T moved into the B operand
 //    with movmatrix.  e4m3 K/V become f16 exactly (bit placement, see
 //    pa_device.cuh), and the 2^8 factor plus the per-tensor scales are folded
 //    into the softmax scale and the output scale.
-//  * At the end of a sequence's range the four warps' states are merged in
-//    shared memory.
 #include <cuda_runtime.h>
 
 #include "pa_device.cuh"
@@ -37,11 +44,10 @@
 namespace pa {
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kGPad = 8;          // query rows per MMA N tile
-constexpr int kMergeStride = 4;   // padding of the merge buffer rows (floats)
-constexpr int kMaxStages = 32;
+constexpr int kWarps = 4;  // compute warps per CTA; each also issues its own loads
+constexpr int kThreads = kWarps * 32;
+constexpr int kGPad = 8;         // query rows per MMA N tile
+constexpr int kMaxStagesPerWarp = 8;
 constexpr int kSmemPerSM = 233472;  // B200: 228 KB per SM
 constexpr int kCtasPerSM = 2;
 
@@ -51,52 +57,80 @@ struct Cfg {
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int ROW = D * ELEM;   // bytes per token row
   static constexpr int TILE = BS * ROW;  // bytes of one K (or V) tile
-  static constexpr int STAGE = 2 * TILE;
+  static constexpr int KVB = 2 * TILE;   // K and V tiles of a stage
   static constexpr int NCH = ROW / 128;  // 128-byte chunks per K/V row
   static constexpr int KM = BS / 16;     // 16-key m-tiles per tile
   static constexpr int DM = D / 16;      // 16-d m-tiles of O^T
-  static constexpr int QROW = D * 2;     // bytes per bf16 query row
   static constexpr int KSTEPS = D / 16;  // k-steps of S^T = K Q^T
   static_assert(ROW % 128 == 0, "rows must be whole 128-byte swizzle rows");
   static_assert(BS % 16 == 0, "block size must be a multiple of 16");
 };
 
 struct SmemLayout {
-  uint32_t ring, qbuf, merge_o, merge_ml, bars, prefix, total;
+  uint32_t ring, bars, info, prefix, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int qrow_bytes, int d, int nstages,
-                                                  int num_seqs) {
+// A stage holds one tile's K and V and, when the tile opens a (sequence, kv
+// head) piece, that piece's query rows (`q_area` bytes, a multiple of 1 KB so
+// the next stage's tiles stay 1 KB aligned for the 128-byte swizzle).
+__host__ __device__ inline int q_area_bytes(int group, int d) { return (group * d * 2 + 1023) / 1024 * 1024; }
+
+__host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int num_seqs) {
   SmemLayout L;
   uint32_t off = 0;
   L.ring = off;
-  off += (uint32_t)stage_bytes * nstages;
-  L.qbuf = off;
-  off += 2u * kGPad * qrow_bytes;
-  L.merge_o = off;
-  off += (uint32_t)kConsumerWarps * kGPad * (d + kMergeStride) * 4;
-  L.merge_ml = off;
-  off += (uint32_t)kConsumerWarps * kGPad * 2 * 4;
+  off += (uint32_t)stage_bytes * nsw * kWarps;
   L.bars = off;
-  off += (uint32_t)(2 * nstages + 4) * 8;
+  off += (uint32_t)kWarps * nsw * 8;
+  L.info = off;
+  off += (uint32_t)kWarps * nsw * 16;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
   return L;
 }
 
+// Tile indices fit in 32 bits (the host rejects batches whose tile count
+// could reach 2^31), so all per-tile arithmetic is 32-bit.
+
 // Largest s in [0, S) with hkv * prefix[s] <= t (that sequence has tiles).
-__device__ __forceinline__ int find_seq(const int32_t* prefix, int S, int hkv, int64_t t) {
+__device__ __forceinline__ int find_seq(const int32_t* prefix, int S, int hkv, int t) {
   int lo = 0, hi = S - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if ((int64_t)hkv * prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    if (hkv * prefix[mid] <= t) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
-__device__ __forceinline__ int64_t range_start(int64_t c, int64_t T, int64_t P) { return c * T / P; }
-__device__ __forceinline__ int64_t cta_of(int64_t x, int64_t T, int64_t P) { return ((x + 1) * P - 1) / T; }
+// CTA c owns tiles [range_start(c), range_start(c + 1)); cta_of(x) is the
+// CTA owning tile x.
+__device__ __forceinline__ int range_start(int c, int T, int P) { return (int)((int64_t)c * T / P); }
+__device__ __forceinline__ int cta_of(int x, int T, int P) { return (int)((((int64_t)x + 1) * P - 1) / T); }
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Arrival counters of cut pieces.  A contributor stores its partial, then
+// lane 0 adds one with release semantics (no result, so no round trip); the
+// merger acquires the count.  Counters start at zero (the workspace contract)
+// and the merger puts its counter back to zero once it has merged.
+__device__ __forceinline__ void count_in_release(unsigned int* cnt) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(cnt) : "memory");
+}
+__device__ __forceinline__ unsigned int load_acquire(const unsigned int* cnt) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+  return v;
+}
 
 template <int KV, int D, int BS>
 __global__ void __launch_bounds__(kThreads, kCtasPerSM)
@@ -105,24 +139,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
   using C = Cfg<KV, D, BS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int NST = p.nstages;
+  const int NSW = p.nstages;  // ring stages per warp
   const int S = p.rows.num_seqs;
-  const SmemLayout L = smem_layout(C::STAGE, C::QROW, D, NST, S);
-  uint8_t* ring = smem + L.ring;
-  uint8_t* qbuf = smem + L.qbuf;
-  float* merge_o = reinterpret_cast<float*>(smem + L.merge_o);
-  float* merge_ml = reinterpret_cast<float*>(smem + L.merge_ml);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + NST;
-  uint64_t* qfull = empty + NST;
-  uint64_t* qempty = qfull + 2;
+  const int hkv = p.num_kv_heads, G = p.group, hq = p.num_q_heads;
+  const int QA = q_area_bytes(G, D);
+  const int STAGE = C::KVB + QA;  // bytes per ring stage
+  const SmemLayout L = smem_layout(STAGE, NSW, S);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L.prefix);
-  __shared__ int32_t warp_tot[kThreads / 32];
-  __shared__ int abort_flag;
+  __shared__ int32_t warp_tot[kWarps];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int hkv = p.num_kv_heads, G = p.group, hq = p.num_q_heads;
 
   // Everything read below may have been produced by the previous kernel in
   // the stream (programmatic dependent launch lets this grid start early).
@@ -162,180 +189,178 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
     }
     if (tid == kThreads - 1) prefix[S] = run;
   }
-  if (tid == 0) {
-    abort_flag = 0;
-    for (int i = 0; i < NST; ++i) {
-      dev::mbar_init(&full[i], 1);
-      dev::mbar_init(&empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      dev::mbar_init(&qfull[i], 1);
-      dev::mbar_init(&qempty[i], kConsumerWarps);
-    }
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * NSW;  // this warp's ring
+  if (lane == 0) {
+    for (int i = 0; i < NSW; ++i) dev::mbar_init(&full[i], 1);
     dev::fence_barrier_init();
-  }
-  // query rows >= G stay zero (the bulk copy fills rows 0..G-1 only)
-  for (int i = tid; i < 2 * kGPad * C::QROW / 16; i += kThreads) {
-    const int row = (i * 16 / C::QROW) % kGPad;
-    if (row >= G) reinterpret_cast<uint4*>(qbuf)[i] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
 
-  const int64_t T = (int64_t)hkv * prefix[S];
-  const int64_t P = gridDim.x;
-  const int64_t cta = blockIdx.x;
-  const int64_t t0 = range_start(cta, T, P), t1 = range_start(cta + 1, T, P);
-  if (cta == 0)
-    for (int i = tid; i <= S; i += kThreads) p.ws.prefix[i] = prefix[i];
+  const int T = hkv * prefix[S];
+  const int W = gridDim.x * kWarps;  // warps of the grid: the workers
+  const int wk = blockIdx.x * kWarps + warp;
+  // a decode row with an empty context attends nothing: zero output
+  for (int s = blockIdx.x; s < S; s += gridDim.x) {
+    const int qlen = p.rows.qsl ? p.rows.qsl[s + 1] - p.rows.qsl[s] : 1;
+    if (qlen == 1 && prefix[s + 1] == prefix[s]) {
+      const int row = p.rows.qsl ? p.rows.qsl[s] : s;
+      for (int i = tid; i < hq * D; i += kThreads)
+        reinterpret_cast<__nv_bfloat16*>(p.out)[(int64_t)row * hq * D + i] = __float2bfloat16_rn(0.f);
+    }
+  }
   dev::grid_dep_launch();
-  if (t0 >= t1) return;
+  const int wbeg = range_start(wk, T, W), wend = range_start(wk + 1, T, W);
+  if (wbeg >= wend) return;  // no CTA-wide synchronisation follows
 
-  if (warp == kConsumerWarps) {
-    // ===================== producer warp: gather through the table ==========
-    if (lane == 0) {
-      dev::prefetch_tmap(&tm_k);
-      if (!C::FP8) dev::prefetch_tmap(&tm_v);
-    }
-    const uint64_t pol = dev::policy_evict_first();
-    const int nblocks = p.max_blocks;
-    int seg_count = 0;
-    bool ok = true;
-    int64_t issued = 0;
-    for (int64_t base = t0; base < t1 && ok; base += 32) {
-      const int64_t t = base + lane;
-      int s = 0, h = 0, blk = 0, row = 0, seg_start = 0;
-      if (t < t1) {
-        s = find_seq(prefix, S, hkv, t);
-        const int nb = prefix[s + 1] - prefix[s];
-        const int64_t local = t - (int64_t)hkv * prefix[s];
-        h = (int)(local / nb);
-        const int i = (int)(local - (int64_t)h * nb);
-        blk = __ldg(p.block_tables + (int64_t)s * nblocks + i);
-        seg_start = (i == 0) || (t == t0);
-        if (seg_start) row = p.rows.qsl ? __ldg(p.rows.qsl + s) : s;
-      }
-      const int cnt = (int)(t1 - base < 32 ? t1 - base : 32);
-      for (int j = 0; j < cnt; ++j) {
-        const int hj = __shfl_sync(0xffffffffu, h, j);
-        int blkj = __shfl_sync(0xffffffffu, blk, j);
-        const int rowj = __shfl_sync(0xffffffffu, row, j);
-        const int ssj = __shfl_sync(0xffffffffu, seg_start, j);
-        if (lane == 0 && ok) {
-          if (blkj < 0 || blkj >= p.num_blocks) {  // bad table entry: flag, read block 0
-            atomicCAS(p.ws.err, 0, 2);
-            blkj = 0;
-          }
-          if (ssj) {
-            const int qb = seg_count & 1;
-            if (seg_count >= 2) ok = dev::mbar_wait(&qempty[qb], ((seg_count >> 1) - 1) & 1, p.ws.err);
-            if (ok) {
-              dev::mbar_arrive_expect_tx(&qfull[qb], (uint32_t)(G * C::QROW));
-              dev::bulk_load(qbuf + qb * kGPad * C::QROW,
-                             p.q + ((int64_t)rowj * hq + (int64_t)hj * G) * C::QROW, (uint32_t)(G * C::QROW),
-                             &qfull[qb], pol);
-            }
-            ++seg_count;
-          }
-          const int64_t k = base + j - t0;
-          const int stage = (int)(k % NST);
-          const uint32_t n = (uint32_t)(k / NST);
-          if (ok && n > 0) ok = dev::mbar_wait(&empty[stage], (n - 1) & 1, p.ws.err);
-          if (ok) {
-            uint8_t* st = ring + (size_t)stage * C::STAGE;
-            dev::mbar_arrive_expect_tx(&full[stage], (uint32_t)C::STAGE);
-            const int32_t krow = (blkj * hkv + hj) * BS;
-#pragma unroll
-            for (int c = 0; c < C::NCH; ++c)
-              dev::tma_load_2d(st + c * BS * 128, &tm_k, c * (128 / C::ELEM), krow, &full[stage], pol);
-            if constexpr (C::FP8) {
-              dev::bulk_load(st + C::TILE, p.v_cache + ((int64_t)blkj * hkv + hj) * C::TILE, (uint32_t)C::TILE,
-                             &full[stage], pol);
-            } else {
-#pragma unroll
-              for (int c = 0; c < C::NCH; ++c)
-                dev::tma_load_2d(st + C::TILE + c * BS * 128, &tm_v, c * 64, krow, &full[stage], pol);
-            }
-            ++issued;
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-      }
-    }
-    if (!ok && lane == 0) {
-      // drain: let copies already issued land before the CTA can exit
-      for (int64_t k = (issued > NST ? issued - NST : 0); k < issued; ++k)
-        dev::mbar_wait(&full[k % NST], (uint32_t)((k / NST) & 1), nullptr, 100000000ull);
-    }
-    return;
+  // ---- this warp's tiles: [wbeg, wend); warp-tile u is tile wbeg + u --------
+  const int nmine = wend - wbeg;
+  uint8_t* ring = smem + L.ring + (size_t)warp * NSW * STAGE;
+  const uint32_t ring_u32 = dev::smem_u32(ring);
+  int4* info = reinterpret_cast<int4*>(smem + L.info) + warp * NSW;  // per stage: query row, length
+  const uint64_t pol = dev::policy_evict_first();
+  if (lane == 0) {
+    dev::prefetch_tmap(&tm_k);
+    if (!C::FP8) dev::prefetch_tmap(&tm_v);
   }
 
-  // ======================= consumer warps ===================================
-  const int g = lane >> 2, tq = lane & 3;
-  const uint32_t ring_u32 = dev::smem_u32(ring);
-  const uint32_t qbuf_u32 = dev::smem_u32(qbuf);
-  const int lr = lane & 7, li = lane >> 3;  // ldmatrix: row within matrix, matrix index
-  // A timed-out wait sets `ok` false: the warp stops waiting and computing,
-  // but still reaches every merge barrier, and all consumer warps leave
-  // together after the barrier that follows (abort_flag), so none is left
-  // waiting on a barrier the others never reach.
-  int64_t t = t0;
-  int seg_count = 0;
-  bool ok = true;
-  while (t < t1) {
-    const int s = find_seq(prefix, S, hkv, t);
-    const int nb = prefix[s + 1] - prefix[s];
-    const int64_t seg0 = (int64_t)hkv * prefix[s];
-    const int h = (int)((t - seg0) / nb);
-    const int64_t a = seg0 + (int64_t)h * nb, b = a + nb;
-    const int64_t pe = min(b, t1);
-    const int len = min(__ldg(p.rows.seq_lens + s), nb * BS);
-    const int row = p.rows.qsl ? __ldg(p.rows.qsl + s) : s;
-
-    // ---- query fragments (B operand of S^T = K Q^T) ----
-    const int qb = seg_count & 1;
-    if (ok) ok = dev::mbar_wait(&qfull[qb], (seg_count >> 1) & 1, p.ws.err);
-    uint32_t qf[C::KSTEPS][2];
-    const uint32_t qrow_u32 = qbuf_u32 + qb * kGPad * C::QROW;
-    if constexpr (!C::FP8) {
-#pragma unroll
-      for (int j = 0; j < C::KSTEPS / 2; ++j)
-        dev::ldsm_x4(qrow_u32 + lr * C::QROW + (4 * j + li) * 16, qf[2 * j][0], qf[2 * j][1], qf[2 * j + 1][0],
-                     qf[2 * j + 1][1]);
-    } else {
-      // d order inside a 16-wide k-step follows the e4m3 byte split: logical
-      // k (2t, 2t+1 | 2t+8, 2t+9) <-> d (4t, 4t+2 | 4t+1, 4t+3)
-      const uint8_t* qr = qbuf + qb * kGPad * C::QROW + g * C::QROW;
-#pragma unroll
-      for (int u = 0; u < C::KSTEPS; ++u) {
-        const uint2 w = *reinterpret_cast<const uint2*>(qr + (16 * u + 4 * tq) * 2);
-        const float q0 = dev::bf16_bits_to_f32(w.x & 0xFFFFu), q1 = dev::bf16_bits_to_f32(w.x >> 16);
-        const float q2 = dev::bf16_bits_to_f32(w.y & 0xFFFFu), q3 = dev::bf16_bits_to_f32(w.y >> 16);
-        qf[u][0] = dev::pack_f16(q0, q2);
-        qf[u][1] = dev::pack_f16(q1, q3);
+  // Lane l of a batch describes warp-tile ub + l: its kv head, physical block
+  // and, if the tile opens a piece, the piece's query row and context length
+  // (row -1 otherwise).  Two batches are kept: the one being issued and the
+  // next one, whose global loads are in flight meanwhile.
+  struct Desc {
+    int h, blk, row, len;
+  };
+  auto describe = [&](int ub) {
+    Desc d{0, 0, -1, 0};
+    const int u = ub + lane;
+    if (u < nmine) {
+      const int t = wbeg + u;
+      const int s = find_seq(prefix, S, hkv, t);
+      const int nb = prefix[s + 1] - prefix[s];
+      const int local = t - hkv * prefix[s];
+      d.h = local / nb;
+      const int i = local - d.h * nb;
+      d.blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + i);
+      if (d.blk < 0 || d.blk >= p.num_blocks) {  // bad table entry: flag, read block 0
+        atomicCAS(p.ws.err, 0, 2);
+        d.blk = 0;
+      }
+      if (i == 0 || t == wbeg) {
+        d.row = p.rows.qsl ? __ldg(p.rows.qsl + s) : s;
+        d.len = min(__ldg(p.rows.seq_lens + s), nb * BS);
       }
     }
+    return d;
+  };
+  int cb = 0;
+  Desc cur = describe(0), nxt{0, 0, -1, 0};
+  // Issue warp-tile u into stage u % NSW (warp-uniform call, u increasing).
+  // A tile that opens a piece also brings the piece's query rows into the
+  // stage's query area, and its row and length into the stage's info slot.
+  auto issue = [&](int u) {
+    if (u >= cb + 32) {
+      cb += 32;
+      cur = nxt;
+      nxt = describe(cb + 32);
+    }
+    const int hj = __shfl_sync(0xffffffffu, cur.h, u - cb);
+    const int blkj = __shfl_sync(0xffffffffu, cur.blk, u - cb);
+    const int rowj = __shfl_sync(0xffffffffu, cur.row, u - cb);
+    const int lenj = __shfl_sync(0xffffffffu, cur.len, u - cb);
+    const int st_i = u % NSW;
+    uint8_t* st = ring + (size_t)st_i * STAGE;
+    const uint32_t qbytes = (uint32_t)(G * D * 2);
+    if (lane == 0) {
+      if (rowj >= 0) info[st_i] = make_int4(rowj, lenj, 0, 0);
+      dev::mbar_arrive_expect_tx(&full[st_i], (uint32_t)C::KVB + (rowj >= 0 ? qbytes : 0u));
+    }
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(&qempty[qb]);
+    // one copy per lane, all in the same instructions: lanes 0..NCH-1 take
+    // the K tile's 128-byte column boxes, the next lanes the V tile, the
+    // next one the query rows
+    const int32_t krow = (blkj * hkv + hj) * BS;
+    if (lane < C::NCH) {
+      dev::tma_load_2d(st + lane * BS * 128, &tm_k, lane * (128 / C::ELEM), krow, &full[st_i], pol);
+    } else if (lane < 2 * C::NCH) {
+      const int c = lane - C::NCH;
+      if constexpr (C::FP8) {
+        dev::bulk_load(st + C::TILE, p.v_cache + ((int64_t)blkj * hkv + hj) * C::TILE, (uint32_t)C::TILE,
+                       &full[st_i], pol);
+      } else {
+        dev::tma_load_2d(st + C::TILE + c * BS * 128, &tm_v, c * 64, krow, &full[st_i], pol);
+      }
+    } else if (lane == 2 * C::NCH && rowj >= 0) {
+      dev::bulk_load(st + C::KVB, p.q + ((int64_t)rowj * hq + (int64_t)hj * G) * D * 2, qbytes, &full[st_i], pol);
+    }
+  };
+  int issued = 0;
+  for (; issued < NSW && issued < nmine; ++issued) issue(issued);
+  nxt = describe(32);  // the next batch, needed from warp-tile 32 on
+
+  const int g = lane >> 2, tq = lane & 3;
+  const int lr = lane & 7, li = lane >> 3;  // ldmatrix: row within matrix, matrix index
+  const int c0 = 2 * tq, c1 = 2 * tq + 1;   // this thread's query columns
+  // A timed-out wait sets `ok` false: the warp stops waiting and computing
+  // and leaves after draining its copies; every wait is bounded.
+  int t = wbeg;
+  int stage = 0;
+  uint32_t phase = 0;
+  int done = 0;  // warp-tiles consumed
+  bool ok = true;
+  while (t < wend && ok) {
+    const int s = find_seq(prefix, S, hkv, t);
+    const int nb = prefix[s + 1] - prefix[s];
+    const int seg0 = hkv * prefix[s];
+    const int h = (t - seg0) / nb;
+    const int a = seg0 + h * nb, b = a + nb;
+    const int pe = min(b, wend);
+    int row = 0, len = 0;
+    uint32_t qf[C::KSTEPS][2];
 
     float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
     float o[C::DM][4];
 #pragma unroll
     for (int i = 0; i < C::DM; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-    for (int64_t tile = t + warp; tile < pe && ok; tile += kConsumerWarps) {
-      const int64_t k = tile - t0;
-      const int stage = (int)(k % NST);
-      ok = dev::mbar_wait(&full[stage], (uint32_t)((k / NST) & 1), p.ws.err);
+    for (int tile = t; ok && tile < pe; ++tile) {
+      ok = __all_sync(0xffffffffu, dev::mbar_wait(&full[stage], phase & 1, p.ws.err));
       if (!ok) break;
-      const uint32_t kbase = ring_u32 + stage * C::STAGE;
+      if (tile == t) {
+        // the piece's first tile: its stage carries the query rows and info
+        const int4 inf = info[stage];
+        row = inf.x;
+        len = inf.y;
+        // ---- query fragments (B operand of S^T = K Q^T), rows >= G are zero ----
+        const uint8_t* qs = ring + (size_t)stage * STAGE + C::KVB + g * D * 2;
+        if constexpr (!C::FP8) {
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            qf[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qs + (16 * kk + 2 * tq) * 2) : 0u;
+            qf[kk][1] = g < G ? *reinterpret_cast<const uint32_t*>(qs + (16 * kk + 2 * tq + 8) * 2) : 0u;
+          }
+        } else {
+          // d order inside a 16-wide k-step follows the e4m3 byte split:
+          // logical k (2t, 2t+1 | 2t+8, 2t+9) <-> d (4t, 4t+2 | 4t+1, 4t+3)
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            uint2 w = make_uint2(0u, 0u);
+            if (g < G) w = *reinterpret_cast<const uint2*>(qs + (16 * kk + 4 * tq) * 2);
+            const float q0 = dev::bf16_bits_to_f32(w.x & 0xFFFFu), q1 = dev::bf16_bits_to_f32(w.x >> 16);
+            const float q2 = dev::bf16_bits_to_f32(w.y & 0xFFFFu), q3 = dev::bf16_bits_to_f32(w.y >> 16);
+            qf[kk][0] = dev::pack_f16(q0, q2);
+            qf[kk][1] = dev::pack_f16(q1, q3);
+          }
+        }
+      }
+      const uint32_t kbase = ring_u32 + stage * STAGE;
       const uint32_t vbase = kbase + C::TILE;
-      const int key0 = (int)(tile - a) * BS;
+      const int key0 = (tile - a) * BS;
       if (len - key0 < BS) {
         // Slots past the context hold whatever the pool last stored there
         // (possibly NaN/Inf bit patterns): their scores are masked to -inf,
         // but 0 * NaN would still poison P*V, so their V rows are zeroed.
         const int valid = len - key0;
-        uint8_t* vt = ring + (size_t)stage * C::STAGE + C::TILE;
+        uint8_t* vt = ring + (size_t)stage * STAGE + C::TILE;
         if constexpr (!C::FP8) {
           for (int i = lane; i < (BS - valid) * C::NCH * 8; i += 32) {
             const int key = valid + i / (C::NCH * 8), rest = i % (C::NCH * 8);
@@ -343,11 +368,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
                 make_uint4(0, 0, 0, 0);
           }
         } else {
-          for (int i = lane; i < D * (BS - valid); i += 32) vt[(i / (BS - valid)) * BS + valid + i % (BS - valid)] = 0;
+          for (int i = lane; i < D * (BS - valid); i += 32)
+            vt[(i / (BS - valid)) * BS + valid + i % (BS - valid)] = 0;
         }
-        // order these generic-proxy writes before the async-proxy (TMA)
-        // writes that refill this stage later
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
       }
 
@@ -470,132 +493,158 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
           }
         }
       }
+      // this stage is consumed: refill it with warp-tile u + NSW.  The
+      // proxy fence orders this warp's generic-proxy accesses to the stage
+      // before the TMA (async proxy) writes into it again.
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&empty[stage]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (issued < nmine) issue(issued++);
+      ++done;
+      if (++stage == NSW) {
+        stage = 0;
+        ++phase;
+      }
     }
-    if (!ok && lane == 0) abort_flag = 1;
+    if (!ok) break;
 
-    // ---- merge the four warps' states for this (sequence, kv head) ----
+    // ---- finish this (sequence, kv head) piece ----
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, off);
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
-    constexpr int MS = D + kMergeStride;
-    float* mo = merge_o + warp * kGPad * MS;
-    float* mml = merge_ml + warp * kGPad * 2;
-    if (g == 0) {
-      mml[(2 * tq) * 2] = m0;
-      mml[(2 * tq) * 2 + 1] = l0;
-      mml[(2 * tq + 1) * 2] = m1;
-      mml[(2 * tq + 1) * 2 + 1] = l1;
-    }
+    const int64_t obase = ((int64_t)row * hq + (int64_t)h * G) * D;
+    if (t == a && pe == b) {
+      // the whole context is in this warp's range: write the output
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + obase;
+      const float i0 = p.out_scale / l0, i1 = p.out_scale / l1;
 #pragma unroll
-    for (int mt = 0; mt < C::DM; ++mt) {
-      const int d0 = 16 * mt + g;
-      mo[(2 * tq) * MS + d0] = o[mt][0];
-      mo[(2 * tq + 1) * MS + d0] = o[mt][1];
-      mo[(2 * tq) * MS + d0 + 8] = o[mt][2];
-      mo[(2 * tq + 1) * MS + d0 + 8] = o[mt][3];
-    }
-    dev::named_bar_sync(1, kConsumerWarps * 32);
-    const bool aborted = *reinterpret_cast<volatile int*>(&abort_flag) != 0;
-    const bool complete = (t == a) && (pe == b);
-    const int64_t slot = 2 * cta + (t == t0 ? 0 : 1);
-    for (int idx = tid; idx < (aborted ? 0 : G * D); idx += kConsumerWarps * 32) {
-      const int jq = idx / D, d = idx - jq * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_ml[(w * kGPad + jq) * 2]);
-      float lsum = 0.f, acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float e = dev::ex2(merge_ml[(w * kGPad + jq) * 2] - M);
-        lsum += merge_ml[(w * kGPad + jq) * 2 + 1] * e;
-        acc += merge_o[(w * kGPad + jq) * MS + d] * e;
-      }
-      if (complete) {
-        const int64_t oi = ((int64_t)row * hq + (int64_t)h * G + jq) * D + d;
-        reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(acc / lsum * p.out_scale);
-      } else {
-        p.ws.o[(slot * G + jq) * D + d] = acc;
-        if (d == 0) {
-          p.ws.ml[(slot * G + jq) * 2] = M;
-          p.ws.ml[(slot * G + jq) * 2 + 1] = lsum;
+      for (int mt = 0; mt < C::DM; ++mt) {
+        const int d0 = 16 * mt + g;
+        if (c0 < G) {
+          out[c0 * D + d0] = __float2bfloat16_rn(o[mt][0] * i0);
+          out[c0 * D + d0 + 8] = __float2bfloat16_rn(o[mt][2] * i0);
+        }
+        if (c1 < G) {
+          out[c1 * D + d0] = __float2bfloat16_rn(o[mt][1] * i1);
+          out[c1 * D + d0 + 8] = __float2bfloat16_rn(o[mt][3] * i1);
         }
       }
+    } else if (t != a) {
+      // a later piece of a sequence cut by warp ranges: store the partial
+      // (this warp's first piece, so slot 2 * wk) and count it in
+      float* po = p.ws.o + 2 * (int64_t)wk * G * D;
+      float* pml = p.ws.ml + 2 * (int64_t)wk * G * 2;
+#pragma unroll
+      for (int mt = 0; mt < C::DM; ++mt) {
+        const int d0 = 16 * mt + g;
+        if (c0 < G) {
+          po[c0 * D + d0] = o[mt][0];
+          po[c0 * D + d0 + 8] = o[mt][2];
+        }
+        if (c1 < G) {
+          po[c1 * D + d0] = o[mt][1];
+          po[c1 * D + d0 + 8] = o[mt][3];
+        }
+      }
+      if (g == 0) {
+        if (c0 < G) {
+          pml[c0 * 2] = m0;
+          pml[c0 * 2 + 1] = l0;
+        }
+        if (c1 < G) {
+          pml[c1 * 2] = m1;
+          pml[c1 * 2 + 1] = l1;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) count_in_release(p.ws.cnt + (int64_t)s * hkv + h);
+    } else {
+      // the sequence's first piece, cut by the end of this warp's range:
+      // this warp merges.  It finishes after the other pieces (they sit at
+      // the starts of later warps' ranges), waits for their count, and folds
+      // their partials into its own state in the MMA fragment layout: a
+      // log-sum-exp combine, then the output.
+      const int cf = wk, cl = cta_of(b - 1, T, W);
+      int others = 0;
+      for (int c = cf + 1; c <= cl; ++c) others += range_start(c, T, W) < range_start(c + 1, T, W);
+      unsigned int* cnt = p.ws.cnt + (int64_t)s * hkv + h;
+      bool ready = true;
+      if (lane == 0) {
+        const uint64_t t_start = dev::globaltimer_ns();
+        while (load_acquire(cnt) < (unsigned)others) {
+          if (dev::globaltimer_ns() - t_start > 2000000000ull) {  // bounded: flag and give up
+            atomicCAS(p.ws.err, 0, 1);
+            ready = false;
+            break;
+          }
+        }
+      }
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      __syncwarp();
+      // running max per query column over this warp and every contributor
+      float M0 = m0, M1 = m1;
+      for (int c = cf + 1; c <= cl && ready; ++c) {
+        if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
+        const float* pml = p.ws.ml + 2 * (int64_t)c * G * 2;
+        if (c0 < G) M0 = fmaxf(M0, __ldcg(pml + c0 * 2));
+        if (c1 < G) M1 = fmaxf(M1, __ldcg(pml + c1 * 2));
+      }
+      const float e0 = dev::ex2(m0 - M0), e1 = dev::ex2(m1 - M1);
+      float L0 = l0 * e0, L1 = l1 * e1;
+#pragma unroll
+      for (int mt = 0; mt < C::DM; ++mt) {
+        o[mt][0] *= e0;
+        o[mt][2] *= e0;
+        o[mt][1] *= e1;
+        o[mt][3] *= e1;
+      }
+      for (int c = cf + 1; c <= cl && ready; ++c) {
+        if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
+        const float* pml = p.ws.ml + 2 * (int64_t)c * G * 2;
+        const float* po = p.ws.o + 2 * (int64_t)c * G * D;
+        const float w0 = c0 < G ? dev::ex2(__ldcg(pml + c0 * 2) - M0) : 0.f;
+        const float w1 = c1 < G ? dev::ex2(__ldcg(pml + c1 * 2) - M1) : 0.f;
+        if (c0 < G) L0 += __ldcg(pml + c0 * 2 + 1) * w0;
+        if (c1 < G) L1 += __ldcg(pml + c1 * 2 + 1) * w1;
+#pragma unroll
+        for (int mt = 0; mt < C::DM; ++mt) {
+          const int d0 = 16 * mt + g;
+          if (c0 < G) {
+            o[mt][0] += w0 * __ldcg(po + c0 * D + d0);
+            o[mt][2] += w0 * __ldcg(po + c0 * D + d0 + 8);
+          }
+          if (c1 < G) {
+            o[mt][1] += w1 * __ldcg(po + c1 * D + d0);
+            o[mt][3] += w1 * __ldcg(po + c1 * D + d0 + 8);
+          }
+        }
+      }
+      // L0/L1 are whole-column sums already: l0/l1 were reduced over the
+      // warp above and a partial's sum is per column
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + obase;
+      const float i0 = p.out_scale / L0, i1 = p.out_scale / L1;
+#pragma unroll
+      for (int mt = 0; mt < C::DM; ++mt) {
+        const int d0 = 16 * mt + g;
+        if (c0 < G) {
+          out[c0 * D + d0] = __float2bfloat16_rn(o[mt][0] * i0);
+          out[c0 * D + d0 + 8] = __float2bfloat16_rn(o[mt][2] * i0);
+        }
+        if (c1 < G) {
+          out[c1 * D + d0] = __float2bfloat16_rn(o[mt][1] * i1);
+          out[c1 * D + d0 + 8] = __float2bfloat16_rn(o[mt][3] * i1);
+        }
+      }
+      // ready for the next call (or a replay of this one)
+      __syncwarp();
+      if (lane == 0 && ready) *cnt = 0u;
     }
-    dev::named_bar_sync(1, kConsumerWarps * 32);
-    if (aborted) return;
     t = pe;
-    ++seg_count;
   }
-}
-
-// Merges the partials of every (sequence, kv head) whose tiles were split
-// over several CTAs: a log-sum-exp combine, one warp per (sequence, kv head),
-// contributors spread over lanes and reduced with warp shuffles.
-template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  dev::grid_dep_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int S = p.rows.num_seqs, hkv = p.num_kv_heads, G = p.group, hq = p.num_q_heads;
-  if (wid >= (int64_t)S * hkv) return;
-  const int s = (int)(wid / hkv), h = (int)(wid % hkv);
-  const int32_t* prefix = p.ws.prefix;
-  const int nb = prefix[s + 1] - prefix[s];
-  const int row = p.rows.qsl ? p.rows.qsl[s] : s;
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-  if (nb == 0) {
-    const int qlen = p.rows.qsl ? p.rows.qsl[s + 1] - p.rows.qsl[s] : 1;
-    if (qlen == 1)  // an empty context attends nothing: zero output
-      for (int jq = 0; jq < G; ++jq)
-        for (int d = lane; d < D; d += 32)
-          out[((int64_t)row * hq + (int64_t)h * G + jq) * D + d] = __float2bfloat16_rn(0.f);
-    return;
-  }
-  const int64_t T = (int64_t)hkv * prefix[S];
-  const int64_t P = p.grid;
-  const int64_t a = (int64_t)hkv * prefix[s] + (int64_t)h * nb, b = a + nb;
-  const int64_t cf = cta_of(a, T, P), cl = cta_of(b - 1, T, P);
-  if (cf == cl) return;  // finished in place by its only CTA
-  constexpr int E = D / 32;
-  for (int jq = 0; jq < G; ++jq) {
-    float M = -INFINITY;
-    for (int64_t c = cf + lane; c <= cl; c += 32) {
-      const int64_t slot = 2 * c + (range_start(c, T, P) < a ? 1 : 0);
-      M = fmaxf(M, p.ws.ml[(slot * G + jq) * 2]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float lsum = 0.f, acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int64_t cb = cf; cb <= cl; cb += 32) {
-      const int64_t c = cb + lane;
-      float w = 0.f;
-      int64_t slot = 0;
-      if (c <= cl) {
-        slot = 2 * c + (range_start(c, T, P) < a ? 1 : 0);
-        w = dev::ex2(p.ws.ml[(slot * G + jq) * 2] - M);
-        lsum += p.ws.ml[(slot * G + jq) * 2 + 1] * w;
-      }
-      const int n = (int)(cl - cb + 1 < 32 ? cl - cb + 1 : 32);
-      for (int k = 0; k < n; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, w, k);
-        const int64_t sk = __shfl_sync(0xffffffffu, slot, k);
-        const float* po = p.ws.o + (sk * G + jq) * D;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] += wk * po[lane + 32 * e];
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    const float inv = p.out_scale / lsum;
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-      out[((int64_t)row * hq + (int64_t)h * G + jq) * D + lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+  if (!ok && lane == 0) {
+    // drain: let this warp's copies still in flight land before exiting
+    for (int k = done; k < issued; ++k) dev::mbar_wait(&full[k % NSW], (uint32_t)((k / NSW) & 1), nullptr, 100000000ull);
   }
 }
 
@@ -603,10 +652,18 @@ template <int KV, int D, int BS>
 cudaError_t launch_instance(const DecodeParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                             cudaStream_t stream) {
   using C = Cfg<KV, D, BS>;
-  const SmemLayout L = smem_layout(C::STAGE, C::QROW, D, p.nstages, p.rows.num_seqs);
+  const SmemLayout L = smem_layout(C::KVB + q_area_bytes(p.group, D), p.nstages, p.rows.num_seqs);
   auto kern = decode_tc_kernel<KV, D, BS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  // raise the kernel's dynamic shared memory limit once per device
+  static int set_for[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev >= 64 || set_for[dev] < (int)L.total) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) set_for[dev] = (int)L.total;
+  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -617,45 +674,37 @@ cudaError_t launch_instance(const DecodeParams& p, const CUtensorMap& tm_k, cons
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tm_k, tm_v, p);
-  if (e != cudaSuccess) return e;
-  const int64_t warps = (int64_t)p.rows.num_seqs * p.num_kv_heads;
-  cudaLaunchConfig_t cc = {};
-  cc.gridDim = dim3((unsigned)((warps + 3) / 4));
-  cc.blockDim = dim3(128);
-  cc.dynamicSmemBytes = 0;
-  cc.stream = stream;
-  cc.attrs = attr;
-  cc.numAttrs = 1;
-  return cudaLaunchKernelEx(&cc, decode_combine_kernel<D>, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm_k, tm_v, p);
 }
 
 }  // namespace
 
 int decode_tc_grid(int num_sms) { return kCtasPerSM * num_sms; }
+int decode_tc_workers(int num_sms) { return kCtasPerSM * num_sms * kWarps; }
 
-size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int num_seqs, int nstages) {
+size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages) {
   const int elem = kv == kFP8 ? 1 : 2;
-  const int stage = 2 * block_size * head_dim * elem;
-  return smem_layout(stage, head_dim * 2, head_dim, nstages, num_seqs).total;
+  const int stage = 2 * block_size * head_dim * elem + q_area_bytes(group, head_dim);
+  return smem_layout(stage, nstages, num_seqs).total;
 }
 
-// Stages that fit two CTAs per SM.
-static int pick_stages(int kv, int head_dim, int block_size, int num_seqs) {
+// Ring stages per warp that fit `ctas` CTAs per SM.
+static int pick_stages(int kv, int head_dim, int block_size, int group, int num_seqs, int ctas) {
   const int elem = kv == kFP8 ? 1 : 2;
-  const int stage = 2 * block_size * head_dim * elem;
-  const int budget = kSmemPerSM / kCtasPerSM - 1024;  // 1 KB per CTA is reserved
-  const int fixed = (int)smem_layout(stage, head_dim * 2, head_dim, 0, num_seqs).total;
-  int n = (budget - fixed) / (stage + 16);
-  if (n > kMaxStages) n = kMaxStages;
+  const int stage = 2 * block_size * head_dim * elem + q_area_bytes(group, head_dim);
+  // 1 KB per CTA is reserved, plus a little static shared memory
+  const int budget = kSmemPerSM / ctas - 1024 - 64;
+  const int fixed = (int)smem_layout(stage, 0, num_seqs).total;
+  int n = (budget - fixed) / (kWarps * (stage + 8 + 16));
+  if (n > kMaxStagesPerWarp) n = kMaxStagesPerWarp;
   return n;
 }
 
-size_t decode_tc_workspace_bytes(int num_seqs, int group, int head_dim, int num_sms) {
-  const size_t P = (size_t)decode_tc_grid(num_sms);
-  size_t off = 256;                                      // error word
-  off += ((size_t)(num_seqs + 1) * 4 + 255) / 256 * 256;  // prefix
-  off += (2 * P * group * 2 * 4 + 255) / 256 * 256;      // (max, sum)
+size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms) {
+  const size_t P = (size_t)decode_tc_grid(num_sms) * kWarps;  // partial slots come in pairs per warp
+  size_t off = 256;                                                  // error word
+  off += ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;  // arrival counters
+  off += (2 * P * group * 2 * 4 + 255) / 256 * 256;                  // (max, sum)
   off += 2 * P * group * head_dim * 4;                   // partial outputs
   return off;
 }
@@ -663,9 +712,16 @@ size_t decode_tc_workspace_bytes(int num_seqs, int group, int head_dim, int num_
 cudaError_t launch_decode_tc(const DecodeParams& p_in, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                              int kv, int head_dim, int block_size, int num_sms, cudaStream_t stream) {
   DecodeParams p = p_in;
-  p.nstages = pick_stages(kv, head_dim, block_size, p.rows.num_seqs);
+  // two CTAs per SM when each warp still gets a double-buffered ring, else
+  // one CTA per SM with a deeper ring (large blocks)
+  int ctas = kCtasPerSM;
+  p.nstages = pick_stages(kv, head_dim, block_size, p.group, p.rows.num_seqs, ctas);
+  if (p.nstages < 2) {
+    ctas = 1;
+    p.nstages = pick_stages(kv, head_dim, block_size, p.group, p.rows.num_seqs, ctas);
+  }
   if (p.nstages < 2) return cudaErrorNotSupported;
-  p.grid = decode_tc_grid(num_sms);
+  p.grid = ctas * num_sms;
   if (kv == kBF16) {
     if (head_dim == 128 && block_size == 16) return launch_instance<kBF16, 128, 16>(p, tm_k, tm_v, stream);
     if (head_dim == 128 && block_size == 32) return launch_instance<kBF16, 128, 32>(p, tm_k, tm_v, stream);

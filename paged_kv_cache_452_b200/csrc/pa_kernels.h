@@ -32,12 +32,12 @@ struct AttnRows {
   int32_t num_rows;
 };
 
-// Workspace carve-up shared by the split-K decode kernel and its combine.
+// Workspace carve-up of the split-K decode kernel.
 struct DecodeWorkspace {
-  int32_t* err;     // error word (first 4 bytes of the caller's buffer)
-  int32_t* prefix;  // [num_seqs + 1] blocks before sequence s (decode rows only)
-  float* ml;        // [2 * grid][G][2] partial (max, sum) per split piece
-  float* o;         // [2 * grid][G][D] partial unnormalised outputs
+  int32_t* err;             // error word (first 4 bytes of the caller's buffer)
+  unsigned int* cnt;        // [num_seqs * num_kv_heads] arrival counters: zero between calls
+  float* ml;                // [2 * workers][G][2] partial (max, sum) per cut piece
+  float* o;                 // [2 * workers][G][D] partial unnormalised outputs
 };
 
 struct DecodeParams {
@@ -59,9 +59,10 @@ struct DecodeParams {
 // kv: kBF16 or kFP8; returns cudaErrorNotSupported for unsupported shapes.
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                              int kv, int head_dim, int block_size, int num_sms, cudaStream_t stream);
-size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int num_seqs, int nstages);
+size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages);
+int decode_tc_workers(int num_sms);
 int decode_tc_grid(int num_sms);
-size_t decode_tc_workspace_bytes(int num_seqs, int group, int head_dim, int num_sms);
+size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms);
 
 struct SimtParams {
   const uint8_t* q;  // [rows][Hq][D] in q dtype

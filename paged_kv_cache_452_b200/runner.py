@@ -74,8 +74,7 @@ def setup(wl, device, write_chunk_tokens: int = 1 << 18) -> DeviceBatch:
     desc = _desc_for(wl)
     k_cache, v_cache = alloc_cache(desc, device, fill=_SENTINEL[desc.kv_dtype])
     staged, staged_tokens = [], 0
-    for s in range(S):
-        k, v = wl.prior_kv(s)
+    for s, (k, v) in enumerate(_draws_in_order(wl, S)):
         c = num_cached[s]
         if k.shape[0] - c > 0:
             staged.append((k[c:].to(device), v[c:].to(device), torch.from_numpy(prior_slots[s]).to(device)))
@@ -112,6 +111,23 @@ def setup(wl, device, write_chunk_tokens: int = 1 << 18) -> DeviceBatch:
         prior_slots=prior_slots, num_cached=num_cached)
     torch.cuda.synchronize(device)
     return batch
+
+
+def _draws_in_order(wl, S, window=None):
+    """wl.prior_kv(s) for s = 0..S-1, drawn on a few host threads ahead of
+    use (the draws are independent per sequence), yielded in order."""
+    import concurrent.futures as cf
+    import os
+    window = window or max(2, min(32, (os.cpu_count() or 4)))
+    with cf.ThreadPoolExecutor(max_workers=window) as ex:
+        futs = {}
+        for s in range(min(window, S)):
+            futs[s] = ex.submit(wl.prior_kv, s)
+        for s in range(S):
+            r = futs.pop(s).result()
+            if s + window < S:
+                futs[s + window] = ex.submit(wl.prior_kv, s + window)
+            yield r
 
 
 def _write_staged(desc, staged, k_cache, v_cache):
