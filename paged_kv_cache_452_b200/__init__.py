@@ -5,7 +5,7 @@ Every function here only marshals arguments (torch tensors -> device
 pointers, the current CUDA stream) and calls the library function of the
 same name; all work runs in the library's CUDA kernels or its C++ block pool.
 Importing fails loudly if libpa.so has not been built
-(``python -m paged_kv_cache_452_b200.build``); there is no fallback.
+(``python paged_kv_cache_452_b200/build.py``); there is no fallback.
 """
 import ctypes
 import math

@@ -1,6 +1,9 @@
 """Build libpa.so (all CUDA kernels for sm_100a plus the host pool) in-tree.
 
-    python -m paged_kv_cache_452_b200.build [--verbose]
+    python paged_kv_cache_452_b200/build.py [--verbose] [--force]
+
+(run by path: importing the package loads libpa.so, which may not exist yet
+or may predate the sources)
 
 nvcc compiles each source to an object under _build/ and links them into
 paged_kv_cache_452_b200/libpa.so (static CUDA runtime, no libcuda link: the

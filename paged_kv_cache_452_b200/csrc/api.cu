@@ -166,9 +166,9 @@ WsCarve carve(void* base, int num_seqs, int num_kv_heads, int group, int head_di
   c.ws.cnt = reinterpret_cast<unsigned int*>(b + off);
   off += ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;
   c.ws.ml = reinterpret_cast<float*>(b + off);
-  off += (2 * P * group * 2 * 4 + 255) / 256 * 256;
+  off += (P * group * 2 * 4 + 255) / 256 * 256;
   c.ws.o = reinterpret_cast<float*>(b + off);
-  off += 2 * P * group * head_dim * 4;
+  off += P * group * head_dim * 4;
   c.bytes = off;
   return c;
 }

@@ -531,10 +531,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
         }
       }
     } else if (t != a) {
-      // a later piece of a sequence cut by warp ranges: store the partial
-      // (this warp's first piece, so slot 2 * wk) and count it in
-      float* po = p.ws.o + 2 * (int64_t)wk * G * D;
-      float* pml = p.ws.ml + 2 * (int64_t)wk * G * 2;
+      // a later piece of a sequence cut by warp ranges (it starts this
+      // warp's range, so each warp has at most one): store the partial in
+      // the warp's slot and count it in
+      float* po = p.ws.o + (int64_t)wk * G * D;
+      float* pml = p.ws.ml + (int64_t)wk * G * 2;
 #pragma unroll
       for (int mt = 0; mt < C::DM; ++mt) {
         const int d0 = 16 * mt + g;
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
       float M0 = m0, M1 = m1;
       for (int c = cf + 1; c <= cl && ready; ++c) {
         if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
-        const float* pml = p.ws.ml + 2 * (int64_t)c * G * 2;
+        const float* pml = p.ws.ml + (int64_t)c * G * 2;
         if (c0 < G) M0 = fmaxf(M0, __ldcg(pml + c0 * 2));
         if (c1 < G) M1 = fmaxf(M1, __ldcg(pml + c1 * 2));
       }
@@ -601,8 +602,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
       }
       for (int c = cf + 1; c <= cl && ready; ++c) {
         if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
-        const float* pml = p.ws.ml + 2 * (int64_t)c * G * 2;
-        const float* po = p.ws.o + 2 * (int64_t)c * G * D;
+        const float* pml = p.ws.ml + (int64_t)c * G * 2;
+        const float* po = p.ws.o + (int64_t)c * G * D;
         const float w0 = c0 < G ? dev::ex2(__ldcg(pml + c0 * 2) - M0) : 0.f;
         const float w1 = c1 < G ? dev::ex2(__ldcg(pml + c1 * 2) - M1) : 0.f;
         if (c0 < G) L0 += __ldcg(pml + c0 * 2 + 1) * w0;
@@ -701,11 +702,11 @@ static int pick_stages(int kv, int head_dim, int block_size, int group, int num_
 }
 
 size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms) {
-  const size_t P = (size_t)decode_tc_grid(num_sms) * kWarps;  // partial slots come in pairs per warp
+  const size_t P = (size_t)decode_tc_workers(num_sms);  // one partial slot per warp
   size_t off = 256;                                                  // error word
   off += ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;  // arrival counters
-  off += (2 * P * group * 2 * 4 + 255) / 256 * 256;                  // (max, sum)
-  off += 2 * P * group * head_dim * 4;                   // partial outputs
+  off += (P * group * 2 * 4 + 255) / 256 * 256;                      // (max, sum)
+  off += P * group * head_dim * 4;                                   // partial outputs
   return off;
 }
 

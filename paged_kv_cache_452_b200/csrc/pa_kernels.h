@@ -36,8 +36,8 @@ struct AttnRows {
 struct DecodeWorkspace {
   int32_t* err;             // error word (first 4 bytes of the caller's buffer)
   unsigned int* cnt;        // [num_seqs * num_kv_heads] arrival counters: zero between calls
-  float* ml;                // [2 * workers][G][2] partial (max, sum) per cut piece
-  float* o;                 // [2 * workers][G][D] partial unnormalised outputs
+  float* ml;                // [workers][G][2] partial (max, sum), one cut piece per warp
+  float* o;                 // [workers][G][D] partial unnormalised outputs
 };
 
 struct DecodeParams {
