@@ -129,6 +129,24 @@ int pa_decode(const pa_cache_desc* desc, const void* q, const void* k_cache, con
               int32_t num_seqs, float scale, void* out, void* workspace, size_t workspace_bytes,
               void* stream);
 
+/* pa_decode_static: pa_decode without a caller workspace, for callers that
+ * cannot allocate device memory (inside a captured CUDA graph where
+ * allocation is not allowed, under another owner's allocator, or on a path
+ * that must not allocate after start-up).  The paper has no counterpart;
+ * this is a convenience of this library.
+ * Same arguments and result as pa_decode, minus the workspace: the scratch
+ * is an 8 MiB area compiled into the library, held by every GPU that loads
+ * it until the process exits.  Batches whose pa_decode_workspace_size
+ * exceeds 8 MiB are rejected with PA_ERR_UNSUPPORTED (use pa_decode).
+ * The first call on a device looks up the area's device address (with that
+ * device current); make that first call before any stream capture.  Every
+ * call clears the area's error word and arrival counters on `stream` first,
+ * so in-kernel error reports are not kept between calls.  All calls share
+ * the one area: calls that overlap on the GPU race.  Allocates nothing. */
+int pa_decode_static(const pa_cache_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                     int32_t num_seqs, float scale, void* out, void* stream);
+
 /* Scratch bytes pa_decode_chunked_prefill needs. */
 size_t pa_prefill_workspace_size(const pa_cache_desc* desc, int32_t num_seqs, int32_t num_tokens);
 

@@ -129,6 +129,15 @@ def pa_decode(desc, q, k_cache, v_cache, block_tables, seq_lens, scale, out, wor
                            _stream(stream)), "pa_decode")
 
 
+def pa_decode_static(desc, q, k_cache, v_cache, block_tables, seq_lens, scale, out, stream=None):
+    """pa_decode without a workspace: the scratch is a fixed 8 MiB area built
+    into the library, for callers that cannot allocate device memory."""
+    s = int(seq_lens.shape[0])
+    _check(lib().pa_decode_static(ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                  int(block_tables.shape[1]), _ptr(seq_lens), s, float(scale), _ptr(out),
+                                  _stream(stream)), "pa_decode_static")
+
+
 def pa_decode_chunked_prefill(desc, q, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
                               max_q_len, scale, out, workspace, stream=None):
     """A mixed step: sequence s owns rows query_start_loc[s]..query_start_loc[s+1]-1 (causal)."""

@@ -17,6 +17,7 @@ SIGNATURES = {
     "pa_cache_write": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _P, _P]),
     "pa_decode_workspace_size": (_SZ, [_P, _I32]),
     "pa_decode": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P, _SZ, _P]),
+    "pa_decode_static": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P]),
     "pa_prefill_workspace_size": (_SZ, [_P, _I32, _I32]),
     "pa_decode_chunked_prefill": (ctypes.c_int,
                                   [_P, _P, _P, _P, _P, _I32, _P, _P, _I32, _I32, _I32, _F, _P, _P, _SZ, _P]),
