@@ -309,7 +309,8 @@ def bench_ours(args):
                      "peak_source": src, "traffic": None, "kernel_ms": attend_ms},
         "e2e": {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+        # pa_cache_write + pa_decode's decode kernel (+ its prefill kernel for prompt rows)
+        "gpu_launches": (3 if int(wl.q_lens.max()) > 1 else 2) * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:

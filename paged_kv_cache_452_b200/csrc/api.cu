@@ -364,10 +364,34 @@ int pa_decode_chunked_prefill(const pa_cache_desc* d, const void* q, const void*
   if (num_tokens == 0) return PA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (use_tc(d)) {
+    // decode rows on the decode kernel, prompt rows on the prefill kernel
     rc = run_decode_tc(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc,
                        num_seqs, num_tokens, scale, out, workspace, workspace_bytes, st, who);
     if (rc) return rc;
     if (max_q_len <= 1) return PA_OK;
+    const int group = d->num_q_heads / d->num_kv_heads;
+    if (prefill_tc_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group)) {
+      CUtensorMap tm_k, tm_v;
+      if ((rc = make_kv_map(&tm_k, k_cache, d->kv_dtype, d))) return rc;
+      if ((rc = make_kv_map(&tm_v, v_cache, d->kv_dtype, d))) return rc;
+      PrefillParams pp = {};
+      pp.q = static_cast<const uint8_t*>(q);
+      pp.out = static_cast<uint8_t*>(out);
+      pp.block_tables = block_tables;
+      pp.max_blocks = max_blocks_per_seq;
+      pp.rows.seq_lens = seq_lens;
+      pp.rows.qsl = query_start_loc;
+      pp.rows.num_seqs = num_seqs;
+      pp.rows.num_rows = num_tokens;
+      pp.num_q_heads = d->num_q_heads;
+      pp.num_kv_heads = d->num_kv_heads;
+      pp.group = group;
+      pp.num_blocks = d->num_blocks;
+      pp.scale_log2 = scale * 1.4426950408889634f;
+      pp.err = static_cast<int32_t*>(workspace);
+      cudaError_t e = launch_prefill_tc(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
+      if (e != cudaErrorNotSupported) return cuda_status(e, who);
+    }
     return run_simt(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc, num_seqs,
                     num_tokens, 1, scale, out, workspace, st, who);
   }

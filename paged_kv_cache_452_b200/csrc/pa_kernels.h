@@ -64,6 +64,22 @@ int decode_tc_workers(int num_sms);
 int decode_tc_grid(int num_sms);
 size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms);
 
+// Prompt rows (q_len > 1) of a mixed step on the tensor-core path.
+struct PrefillParams {
+  const uint8_t* q;  // bf16 [rows][Hq][D]
+  uint8_t* out;      // bf16 [rows][Hq][D]
+  const int32_t* block_tables;
+  int32_t max_blocks;
+  AttnRows rows;  // qsl required
+  int32_t num_q_heads, num_kv_heads, group, num_blocks;
+  int32_t nstages;
+  float scale_log2;
+  int32_t* err;  // workspace error word
+};
+bool prefill_tc_supported(int kv, int q, int head_dim, int block_size, int group);
+cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                              int head_dim, int block_size, int num_tokens, cudaStream_t stream);
+
 struct SimtParams {
   const uint8_t* q;  // [rows][Hq][D] in q dtype
   uint8_t* out;

@@ -121,10 +121,26 @@ def test_edge_cases(case, cuda_device):
     run_and_check(W.custom(case, **EDGE[case]), cuda_device)
 
 
-def test_mixed_edge_cases(cuda_device):
+MIXED_EDGE = {
     # prefill chunks with no prior context, a 1-token chunk, chunks crossing blocks
-    wl = W.custom("mixed_edges", context_lens=[0, 0, 17, 40, 3, 100], q_lens=[1, 20, 33, 1, 16, 1])
-    run_and_check(wl, cuda_device)
+    "mixed_edges": dict(context_lens=[0, 0, 17, 40, 3, 100], q_lens=[1, 20, 33, 1, 16, 1]),
+    # chunks of exactly one, one less and one more than a unit of query
+    # positions (64 rows / group 4 = 16 positions), over prior context that
+    # ends mid-block and on a block edge
+    "unit_bounds_g4": dict(context_lens=[0, 5, 16, 31, 7], q_lens=[16, 15, 17, 48, 1]),
+    "mha_prefill": dict(context_lens=[3, 70, 0], q_lens=[64, 65, 130], num_q_heads=2, num_kv_heads=2),
+    "group8_prefill": dict(context_lens=[0, 21, 9], q_lens=[8, 9, 40], num_q_heads=16, num_kv_heads=2),
+    "group16_prefill": dict(context_lens=[0, 33], q_lens=[5, 37], num_q_heads=32, num_kv_heads=2),
+    "head64_bs32_prefill": dict(context_lens=[0, 50, 7], q_lens=[70, 3, 1], head_dim=64, block_size=32),
+    "group3_prefill": dict(context_lens=[4, 0], q_lens=[9, 22], num_q_heads=6, num_kv_heads=2),  # CUDA cores
+    "prefill_only": dict(context_lens=[0, 200], q_lens=[33, 100]),
+    "fp8_prefill": dict(context_lens=[0, 40], q_lens=[17, 30], kv_dtype="e4m3"),  # CUDA cores
+}
+
+
+@pytest.mark.parametrize("case", sorted(MIXED_EDGE))
+def test_mixed_edge_cases(case, cuda_device):
+    run_and_check(W.custom(case, **MIXED_EDGE[case]), cuda_device)
 
 
 def test_paged_output_equals_contiguous_output(cuda_device):
@@ -197,6 +213,18 @@ def test_context_longer_than_table_row_is_flagged(cuda_device):
     runner.attend(b)
     torch.cuda.synchronize()
     assert pa.workspace_error(b.workspace) == 3
+
+
+def test_bad_table_entry_in_prompt_rows_is_flagged(cuda_device):
+    wl = W.mixed_prefill(16, "small")
+    b = runner.setup(wl, cuda_device)
+    runner.step(b)
+    torch.cuda.synchronize()
+    assert pa.workspace_error(b.workspace) == 0
+    b.tables[0, 0] = -1  # sequence 0 is a prefill chunk
+    runner.attend(b)
+    torch.cuda.synchronize()
+    assert pa.workspace_error(b.workspace) == 2
 
 
 FULL = [("gqa_bf16", None), ("prefix_bf16", [0, 1, 2, 127, 128, 129, 200, 255]), ("fp8_long", [0, 77]),
