@@ -113,6 +113,18 @@ EDGE = {
     "fewer_tiles_than_ctas": dict(context_lens=[100, 3, 250], num_q_heads=4, num_kv_heads=1),
     "many_short": dict(context_lens=list(range(0, 700, 1)), num_q_heads=4, num_kv_heads=2, head_dim=64),
     "single": dict(context_lens=[1]),
+    # batches with several tiles per worker warp, so contexts are cut at many
+    # warp-range edges and merged from several pieces
+    "split_uniform": dict(context_lens=[2000] * 20, num_q_heads=32, num_kv_heads=8),
+    "split_ragged": dict(context_lens=[0, 1, 17, 3000, 5, 16, 4000, 33, 2500, 1, 64, 6000, 15, 31, 700],
+                       num_q_heads=32, num_kv_heads=8),
+    "split_group8_head64": dict(context_lens=[7999, 8000, 8001, 100, 7000, 8192], num_q_heads=16, num_kv_heads=2,
+                              head_dim=64),
+    "split_fp8": dict(context_lens=[3000] * 15 + [17], kv_dtype="e4m3", num_q_heads=32, num_kv_heads=8),
+    "split_bs32": dict(context_lens=[4000] * 9 + [31, 32, 33], num_q_heads=32, num_kv_heads=8, block_size=32),
+    # groups whose (max, sum) block is not a multiple of 16 bytes
+    "split_group3": dict(context_lens=[5000] * 8 + [3, 40], num_q_heads=6, num_kv_heads=2),
+    "split_group7_head64": dict(context_lens=[5000] * 8 + [0, 16], num_q_heads=14, num_kv_heads=2, head_dim=64),
 }
 
 

@@ -18,9 +18,14 @@ pytestmark = pytest.mark.gpu
 TOL = {"bf16": 2e-2, "e4m3": 6e-2, "f32": 1e-4}
 
 
-@pytest.mark.parametrize("name", ["gqa_bf16", "fp8_long", "prefix_bf16"])
+# group 8 over 6016 tiles: the largest partial slots, contexts cut at many
+# warp-range edges (still within the 8 MiB area)
+GROUP8 = dict(context_lens=[3000] * 16, num_q_heads=16, num_kv_heads=2)
+
+
+@pytest.mark.parametrize("name", ["gqa_bf16", "fp8_long", "prefix_bf16", "group8"])
 def test_static_scratch_matches_workspace_path(name, cuda_device):
-    wl = W.make(name, "small")
+    wl = W.custom(name, **GROUP8) if name == "group8" else W.make(name, "small")
     b = runner.setup(wl, cuda_device)
     runner.step(b)  # pa_cache_write + pa_decode with a caller workspace
     torch.cuda.synchronize()
