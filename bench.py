@@ -131,15 +131,26 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(args):
+def dist_setup(args, backend=None):
+    """One process per GPU, launched by torchrun (RANK / LOCAL_RANK /
+    WORLD_SIZE / MASTER_* from the environment).  Replicas only: the process
+    group carries the start/stop barriers and the max-over-ranks of the
+    timings, never the data path."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.distributed.init_process_group("nccl" if args.impl == "ours" else "gloo",
-                                             timeout=datetime.timedelta(seconds=120))
+        if backend is None:
+            backend = "nccl" if args.impl == "ours" else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def job_throughput(world, bytes_per_replica, ms):
+    """Whole-job GB/s: every rank streamed `bytes_per_replica` per step and
+    the step took `ms` (the max over ranks)."""
+    return world * bytes_per_replica / (ms * 1e-3) / 1e9
 
 
 def reduce_max(x, world, device):
@@ -197,7 +208,9 @@ def cpu_baseline(wl, budget_s=15.0):
 
 def bench_reference(args):
     world, rank, _ = dist_setup(args)
-    if rank != 0:
+    if rank != 0:  # the oracle runs once, on rank 0's host cores
+        if world > 1:
+            torch.distributed.destroy_process_group()
         return
     wl = W.make(args.workload, "full")
     if wl.kv_dtype == "e4m3":
@@ -217,6 +230,8 @@ def bench_reference(args):
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
 
 
 def _time(fn, steps, stream):
@@ -314,7 +329,7 @@ def bench_ours(args):
     hbm = float(peaks["hbm_gbs"])
     achieved = alg_bytes / (attend_ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC, "value": world * alg_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "metric": METRIC, "value": job_throughput(world, alg_bytes, ms), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.kv_dtype if wl.kv_dtype != "e4m3" else "fp8_e4m3",
         "data": "synthetic",
@@ -330,7 +345,7 @@ def bench_ours(args):
         "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (pa_decode)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src, "traffic": profiled_traffic(wl.name), "kernel_ms": attend_ms},
-        "e2e": {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": job_throughput(world, alg_bytes, e2e_ms), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         # pa_cache_write + pa_decode's decode kernel (+ its prefill kernel for prompt rows)
         "gpu_launches": (3 if int(wl.q_lens.max()) > 1 else 2) * args.steps,
