@@ -370,7 +370,8 @@ int pa_decode_chunked_prefill(const pa_cache_desc* d, const void* q, const void*
     if (rc) return rc;
     if (max_q_len <= 1) return PA_OK;
     const int group = d->num_q_heads / d->num_kv_heads;
-    if (prefill_tc_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group)) {
+    const bool umma = prefill_umma_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group);
+    if (umma || prefill_tc_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group)) {
       CUtensorMap tm_k, tm_v;
       if ((rc = make_kv_map(&tm_k, k_cache, d->kv_dtype, d))) return rc;
       if ((rc = make_kv_map(&tm_v, v_cache, d->kv_dtype, d))) return rc;
@@ -389,7 +390,10 @@ int pa_decode_chunked_prefill(const pa_cache_desc* d, const void* q, const void*
       pp.num_blocks = d->num_blocks;
       pp.scale_log2 = scale * 1.4426950408889634f;
       pp.err = static_cast<int32_t*>(workspace);
-      cudaError_t e = launch_prefill_tc(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
+      cudaError_t e = cudaErrorNotSupported;
+      if (umma) e = launch_prefill_umma(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
+      if (e == cudaErrorNotSupported && prefill_tc_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group))
+        e = launch_prefill_tc(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
       if (e != cudaErrorNotSupported) return cuda_status(e, who);
     }
     return run_simt(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc, num_seqs,

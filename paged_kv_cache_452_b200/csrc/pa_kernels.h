@@ -77,6 +77,11 @@ struct PrefillParams {
   int32_t* err;  // workspace error word
 };
 bool prefill_tc_supported(int kv, int q, int head_dim, int block_size, int group);
+// The same rows on tcgen05 (TMEM accumulators); cudaErrorNotSupported when
+// the shape or the batch's unit table does not fit (the caller falls back).
+bool prefill_umma_supported(int kv, int q, int head_dim, int block_size, int group);
+cudaError_t launch_prefill_umma(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                int head_dim, int block_size, int num_tokens, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                               int head_dim, int block_size, int num_tokens, cudaStream_t stream);
 
