@@ -391,7 +391,9 @@ int pa_decode_chunked_prefill(const pa_cache_desc* d, const void* q, const void*
       pp.scale_log2 = scale * 1.4426950408889634f;
       pp.err = static_cast<int32_t*>(workspace);
       cudaError_t e = cudaErrorNotSupported;
-      if (umma) e = launch_prefill_umma(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
+      int sms = 0;
+      if ((rc = num_sms(&sms))) return rc;
+      if (umma) e = launch_prefill_umma(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, sms, st);
       if (e == cudaErrorNotSupported && prefill_tc_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group))
         e = launch_prefill_tc(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
       if (e != cudaErrorNotSupported) return cuda_status(e, who);

@@ -72,7 +72,8 @@ struct PrefillParams {
   int32_t max_blocks;
   AttnRows rows;  // qsl required
   int32_t num_q_heads, num_kv_heads, group, num_blocks;
-  int32_t nstages;
+  int32_t nstages;    // ring stages (the tcgen05 kernel: K stages)
+  int32_t nstages_v;  // the tcgen05 kernel's V stages
   float scale_log2;
   int32_t* err;  // workspace error word
 };
@@ -81,7 +82,7 @@ bool prefill_tc_supported(int kv, int q, int head_dim, int block_size, int group
 // the shape or the batch's unit table does not fit (the caller falls back).
 bool prefill_umma_supported(int kv, int q, int head_dim, int block_size, int group);
 cudaError_t launch_prefill_umma(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                int head_dim, int block_size, int num_tokens, cudaStream_t stream);
+                                int head_dim, int block_size, int num_tokens, int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                               int head_dim, int block_size, int num_tokens, cudaStream_t stream);
 

@@ -8,20 +8,27 @@
 // the step() list: a step schedules decode and chunked prefill together; the
 // chunk's K/V are already in the pool).
 //
-// How: one CTA per unit = (sequence, kv head, 128 / G query positions).  The
-// GQA group's heads of each position fill the MMA's M = 128 rows, so every
-// K/V tile serves all of them.
-//  * warp 0 walks the block table and brings 128-key K/V tiles into a ring of
-//    shared-memory stages with TMA (2-D boxes of [block][128 B], 128-byte
-//    swizzle, boxes of consecutive blocks stacked into one swizzled tile);
-//    blocks past the keys the unit needs are read out of range, which TMA
-//    fills with zeros;
+// How: a unit = (sequence, kv head, 128 / G query positions); the GQA
+// group's heads of each position fill the MMA's M = 128 rows, so every K/V
+// tile serves all of them.  One persistent CTA per SM walks its share of the
+// units; the rings, the S buffers and the barriers run on across units, so
+// the next unit's first tiles load while the current one finishes.
+//  * warps 0 and 10 walk the block table and bring the K and the V halves of
+//    128-key tiles into two rings of shared-memory stages with TMA (2-D
+//    boxes of [block][128 B], 128-byte swizzle, boxes of consecutive blocks
+//    stacked into one swizzled tile); a K stage is free again as soon as its
+//    S MMA has run, a V stage once its PV MMA has; blocks past the keys the
+//    unit needs are read out of range, which TMA fills with zeros; table
+//    entries are read one tile ahead;
 //  * warp 1 holds the TMEM allocation and, from one thread, issues
 //    S = Q K^T (M 128, N 128, K 16 steps; double-buffered S in TMEM) and
 //    O += P V (N = head_dim; O stays in TMEM across tiles), committing each
-//    to an mbarrier;
-//  * warps 2..5 own one query row per thread: they read the row of S from
-//    TMEM, mask (causal, context length), keep a running max reference that
+//    to an mbarrier; PV of a tile goes out as soon as its P is written, the
+//    S two tiles ahead after it;
+//  * warps 2..9 own half a query row per thread (two warps per TMEM lane
+//    quarter, so two per SM sub-partition): they read their 64 keys of the
+//    row of S from TMEM, mask (causal, context length), combine the row's max
+//    with the other half through shared memory, keep a running max reference that
 //    moves only when the row's max grows by more than 2^8 (then the row of
 //    O in TMEM and the running sum are rescaled: the result is unchanged,
 //    the rescale is rare), write P = 2^(s - ref) as bf16 into a swizzled
@@ -38,7 +45,8 @@ namespace {
 
 constexpr int kRows = 128;    // query rows per unit (positions x group): the MMA's M
 constexpr int kKeys = 128;    // keys per K/V tile: N of S = Q K^T, K of O = P V
-constexpr int kThreads = 192;  // warp 0 loads, warp 1 issues MMAs, warps 2..5 one row per thread
+constexpr int kThreads = 352;  // warps 0/10 load K/V, warp 1 issues MMAs, warps 2..9 half a row per thread
+constexpr int kRowWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemOptIn = 232448;  // 227 KB per block
 constexpr int kChunk = 128 * 128;   // one 128-byte-wide chunk of a 128-row tile
@@ -48,43 +56,50 @@ template <int D, int BS>
 struct U {
   static constexpr int NCH = D / 64;               // 128-byte chunks of a row
   static constexpr int QBYTES = NCH * kChunk;      // Q tile
-  static constexpr int KVT = NCH * kChunk;         // K (or V) tile
-  static constexpr int STAGE = 2 * KVT;
+  static constexpr int KVT = NCH * kChunk;         // K (or V) tile: one ring stage
   static constexpr int BPT = kKeys / BS;           // blocks per tile
-  static constexpr int BOXES = 2 * NCH * BPT;      // TMA boxes per stage
+  static constexpr int BOXES = NCH * BPT;          // TMA boxes per stage
   static constexpr int KSTEPS_S = D / 16;
   static constexpr int KSTEPS_O = kKeys / 16;
-  static_assert(BOXES <= 32, "one box per producer lane");
+  static_assert(BOXES <= 32, "one box per loader lane");
 };
 
 struct Bars {
-  // ring: full[i], empty[i]; then s_full[2], s_free[2], p_full, o_full, q_full, done
-  uint64_t* full;
-  uint64_t* empty;
+  // kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], then s_full[2],
+  // s_free[2], p_full, o_full, q_full, o_free, done
+  uint64_t* kfull;
+  uint64_t* kempty;
+  uint64_t* vfull;
+  uint64_t* vempty;
   uint64_t* s_full;
   uint64_t* s_free;
   uint64_t* p_full;
   uint64_t* o_full;
   uint64_t* q_full;
+  uint64_t* o_free;
   uint64_t* done;
 };
 
 struct ULayout {
-  uint32_t q, p, ring, bars, tmem, prefix, total;
+  uint32_t q, p, kring, vring, bars, tmem, xch, prefix, total;
 };
-__host__ __device__ inline ULayout u_layout(int qbytes, int stage, int nst, int num_seqs) {
+__host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int nsv, int num_seqs) {
   ULayout L;
   uint32_t off = 0;
   L.q = off;
   off += qbytes;
   L.p = off;
   off += 2 * kChunk;
-  L.ring = off;
-  off += (uint32_t)stage * nst;
+  L.kring = off;
+  off += (uint32_t)kvt * nsk;
+  L.vring = off;
+  off += (uint32_t)kvt * nsv;
   L.bars = off;
-  off += (uint32_t)(2 * nst + 8) * 8;
+  off += (uint32_t)(2 * nsk + 2 * nsv + 9) * 8;
   L.tmem = off;
   off += 16;
+  L.xch = off;  // row max halves [2 tile parities][2 halves][128 rows], row sum halves [2][128]
+  off += (2 * 2 * 128 + 2 * 128) * 4;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
@@ -101,15 +116,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = U<D, BS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int NST = p.nstages;
+  const int NSK = p.nstages, NSV = p.nstages_v;
   const int S = p.rows.num_seqs;
-  const ULayout L = u_layout(C::QBYTES, C::STAGE, NST, S);
+  const ULayout L = u_layout(C::QBYTES, C::KVT, NSK, NSV, S);
   uint8_t* qs = smem + L.q;
   uint8_t* ps = smem + L.p;
-  uint8_t* ring = smem + L.ring;
+  uint8_t* kring = smem + L.kring;
+  uint8_t* vring = smem + L.vring;
   uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L.bars);
-  Bars B{bar0, bar0 + NST, bar0 + 2 * NST, bar0 + 2 * NST + 2, bar0 + 2 * NST + 4, bar0 + 2 * NST + 5,
-         bar0 + 2 * NST + 6, bar0 + 2 * NST + 7};
+  uint64_t* bx = bar0 + 2 * NSK + 2 * NSV;
+  Bars B{bar0, bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 5, bx + 6, bx + 7, bx + 8};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L.prefix);  // units before sequence s
   __shared__ int32_t warp_tot[kThreads / 32];
@@ -149,47 +165,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   dev::grid_dep_launch();
   const int nunits = prefix[S] * hkv;
-  if ((int)blockIdx.x >= nunits) return;  // surplus CTA: nothing allocated yet
+  if ((int)blockIdx.x >= nunits) return;  // nothing allocated yet
 
-  // ---- this CTA's unit: ordinal i / Hkv (a sequence's last query blocks
-  // first), kv head i % Hkv ------------------------------------------------------
-  int s = 0;
-  {
-    const int ub = blockIdx.x / hkv;
+  // Units are processed persistently: this CTA takes ordinals blockIdx.x,
+  // blockIdx.x + gridDim.x, ...  Ordinal i is query block i / Hkv (a
+  // sequence's last query blocks first) of kv head i % Hkv.
+  struct Unit {
+    int s, h, first, q0, qn, pos0, seq_len, nbneed, ntiles;
+  };
+  auto unit_of = [&](int idx) {
+    Unit u;
+    const int ub = idx / hkv;
     int lo = 0, hi = S - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (prefix[mid] <= ub) lo = mid; else hi = mid - 1;
     }
-    s = lo;
-  }
-  const int h = blockIdx.x % hkv;
-  const int nqb = prefix[s + 1] - prefix[s];
-  const int qb = nqb - 1 - (blockIdx.x / hkv - prefix[s]);
-  const int first = p.rows.qsl[s];
-  const int qlen = p.rows.qsl[s + 1] - first;
-  const int seq_len = p.rows.seq_lens[s];
-  const int pos0 = seq_len - qlen;  // position of the sequence's first query row
-  const int q0 = qb * QB;           // first query (local index) of the unit
-  const int qn = min(QB, qlen - q0);
-  const int kend = min(seq_len, pos0 + q0 + qn);  // keys the unit needs: [0, kend)
-  int nbneed = (kend + BS - 1) / BS;
-  if (nbneed > p.max_blocks) {
-    if (tid == 0) atomicCAS(p.err, 0, 3);
-    nbneed = p.max_blocks;
-  }
-  const int ntiles = (nbneed * BS + kKeys - 1) / kKeys;
+    u.s = lo;
+    u.h = idx % hkv;
+    const int qb = prefix[lo + 1] - prefix[lo] - 1 - (ub - prefix[lo]);
+    u.first = p.rows.qsl[lo];
+    const int qlen = p.rows.qsl[lo + 1] - u.first;
+    u.seq_len = p.rows.seq_lens[lo];
+    u.pos0 = u.seq_len - qlen;  // position of the sequence's first query row
+    u.q0 = qb * QB;             // first query (local index) of the unit
+    u.qn = min(QB, qlen - u.q0);
+    const int kend = min(u.seq_len, u.pos0 + u.q0 + u.qn);  // keys the unit needs: [0, kend)
+    u.nbneed = (kend + BS - 1) / BS;
+    if (u.nbneed > p.max_blocks) {
+      if (warp == 2 && lane == 0) atomicCAS(p.err, 0, 3);  // (one reporter)
+      u.nbneed = p.max_blocks;
+    }
+    u.ntiles = (u.nbneed * BS + kKeys - 1) / kKeys;
+    return u;
+  };
 
   if (tid == 0) {
     // one arrival (a TMA transaction or an MMA commit), or one per row warp
-    for (int i = 0; i < 2 * NST; ++i) dev::mbar_init(&bar0[i], 1);
+    for (int i = 0; i < 2 * NSK + 2 * NSV; ++i) dev::mbar_init(&bar0[i], 1);
     for (int i = 0; i < 2; ++i) {
       dev::mbar_init(&B.s_full[i], 1);
-      dev::mbar_init(&B.s_free[i], 4);
+      dev::mbar_init(&B.s_free[i], kRowWarps);
     }
-    dev::mbar_init(B.p_full, 4);
+    dev::mbar_init(B.p_full, kRowWarps);
     dev::mbar_init(B.o_full, 1);
-    dev::mbar_init(B.q_full, 4);
+    dev::mbar_init(B.q_full, kRowWarps);
+    dev::mbar_init(B.o_free, kRowWarps);
     dev::mbar_init(B.done, 1);
     dev::fence_barrier_init();
   }
@@ -202,92 +223,111 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t t_s0 = tbase, t_o = tbase + 2 * kKeys;  // S buffers at columns 0 and 128, O at 256
+  // Tiles are counted over all of this CTA's units ("g"): ring stages,
+  // S buffers and the per-tile barriers' phases follow that count.
 
-  if (warp == 0) {
-    // ======================= loads: K/V tiles through the block table ========
+  if (warp == 0 || warp == 10) {
+    // ======================= loads: the K (warp 0) or V (warp 10) ring ========
+    const bool is_v = warp == 10;
+    const int nsr = is_v ? NSV : NSK;
+    uint64_t* fullb = is_v ? B.vfull : B.kfull;
+    uint64_t* emptyb = is_v ? B.vempty : B.kempty;
+    uint8_t* ringb = is_v ? vring : kring;
+    const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
     const uint64_t pol = dev::policy_evict_last();  // the sequence's other units read the same tiles
     const int32_t oob_row = p.num_blocks * hkv * BS;  // past the pool: TMA fills zeros
+    const int c = lane / C::BPT, j = lane % C::BPT;   // this lane's box: 128-byte chunk, block in tile
+    // this lane's table entry for tile k of unit u (-2: past the needed
+    // blocks); the check waits until the entry is used, so the load overlaps
+    // a tile
+    auto entry = [&](const Unit& u, int k) -> int32_t {
+      const int b = k * C::BPT + j;
+      return (lane < C::BOXES && b < u.nbneed) ? __ldg(p.block_tables + (int64_t)u.s * p.max_blocks + b) : -2;
+    };
     bool ok = true;
-    int k = 0;
-    for (; k < ntiles && ok; ++k) {
-      const int st = k % NST;
-      if (k >= NST) ok = __all_sync(0xffffffffu, dev::mbar_wait(&B.empty[st], ((k / NST) - 1) & 1, p.err));
-      if (!ok) break;
-      int32_t y = oob_row;
-      int kv = 0, c = 0, j = 0;
-      if (lane < C::BOXES) {
-        kv = lane / (C::NCH * C::BPT);
-        c = (lane / C::BPT) % C::NCH;
-        j = lane % C::BPT;
-        const int b = k * C::BPT + j;
-        if (b < nbneed) {
-          int blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + b);
+    int g = 0;
+    for (int idx = blockIdx.x; idx < nunits && ok; idx += gridDim.x) {
+      const Unit u = unit_of(idx);
+      int32_t enext = entry(u, 0);
+      for (int k = 0; k < u.ntiles && ok; ++k, ++g) {
+        const int st = g % nsr;
+        if (g >= nsr) ok = __all_sync(0xffffffffu, dev::mbar_wait(&emptyb[st], ((g / nsr) - 1) & 1, p.err));
+        if (!ok) break;
+        int32_t blk = enext;
+        if (k + 1 < u.ntiles) enext = entry(u, k + 1);
+        int32_t y = oob_row;
+        if (blk != -2) {
           if (blk < 0 || blk >= p.num_blocks) {  // bad table entry: flag, read block 0
             atomicCAS(p.err, 0, 2);
             blk = 0;
           }
-          y = (blk * hkv + h) * BS;
+          y = (blk * hkv + u.h) * BS;
         }
-      }
-      if (lane == 0) dev::mbar_arrive_expect_tx(&B.full[st], (uint32_t)C::STAGE);
-      __syncwarp();
-      if (lane < C::BOXES) {
-        uint8_t* dst = ring + (size_t)st * C::STAGE + kv * C::KVT + c * kChunk + j * BS * 128;
-        dev::tma_load_2d(dst, kv ? &tm_v : &tm_k, c * 64, y, &B.full[st], pol);
+        if (lane == 0) dev::mbar_arrive_expect_tx(&fullb[st], (uint32_t)C::KVT);
+        __syncwarp();
+        if (lane < C::BOXES)
+          dev::tma_load_2d(ringb + (size_t)st * C::KVT + c * kChunk + j * BS * 128, tm, c * 64, y, &fullb[st], pol);
       }
     }
     // drain: the last stages issued must land before this CTA may exit
     if (lane == 0) {
-      for (int d = max(0, k - NST); d < k; ++d)
-        dev::mbar_wait(&B.full[d % NST], (uint32_t)((d / NST) & 1), nullptr, 100000000ull);
+      for (int d = max(0, g - nsr); d < g; ++d)
+        dev::mbar_wait(&fullb[d % nsr], (uint32_t)((d / nsr) & 1), nullptr, 100000000ull);
     }
   } else if (warp == 1) {
     // ======================= MMA issue (one thread) ===========================
     if (lane == 0) {
       const uint32_t idesc_s = dev::umma_idesc_bf16(kKeys, false);
       const uint32_t idesc_o = dev::umma_idesc_bf16(D, true);
-      const uint32_t q_u32 = dev::smem_u32(qs), p_u32 = dev::smem_u32(ps), ring_u32 = dev::smem_u32(ring);
-      auto issue_s = [&](int k) {  // S[k & 1] = Q K_k^T
-        const uint32_t kb = ring_u32 + (uint32_t)((k % NST) * C::STAGE);
+      // descriptors built once; an MMA adds its byte offset / 16 to the
+      // start-address field (addresses stay below 256 KB: no carry out)
+      const uint64_t dq = dev::umma_desc_sw128(dev::smem_u32(qs), 16, 1024);
+      const uint64_t dp = dev::umma_desc_sw128(dev::smem_u32(ps), 16, 1024);
+      const uint64_t dk = dev::umma_desc_sw128(dev::smem_u32(kring), 16, 1024);
+      const uint64_t dv = dev::umma_desc_sw128(dev::smem_u32(vring), kChunk, 1024);
+      // S[g & 1] = Q K_g^T once K_g has landed and S[g & 1]'s last reader is done
+      auto issue_s = [&](int g) -> bool {
+        if (!dev::mbar_wait(&B.kfull[g % NSK], (uint32_t)((g / NSK) & 1), p.err)) return false;
+        if (g >= 2 && !dev::mbar_wait(&B.s_free[g & 1], (uint32_t)(((g >> 1) - 1) & 1), p.err)) return false;
+        dev::tc_fence_after();
+        const uint64_t kb = dk + (uint64_t)(((g % NSK) * C::KVT) >> 4);
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS_S; ++ks) {
-          const uint32_t off = (uint32_t)((ks >> 2) * kChunk + (ks & 3) * 32);
-          dev::umma_ss(t_s0 + (uint32_t)((k & 1) * kKeys), dev::umma_desc_sw128(q_u32 + off, 16, 1024),
-                       dev::umma_desc_sw128(kb + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((ks >> 2) * kChunk + (ks & 3) * 32) >> 4);
+          dev::umma_ss(t_s0 + (uint32_t)((g & 1) * kKeys), dq + off, kb + off, idesc_s, ks > 0 ? 1u : 0u);
         }
-        dev::umma_commit(&B.s_full[k & 1]);
+        dev::umma_commit(&B.s_full[g & 1]);
+        dev::umma_commit(&B.kempty[g % NSK]);
+        return true;
       };
-      bool ok = dev::mbar_wait(B.q_full, 0, p.err);
-      if (ok && ntiles > 0) {
-        ok = dev::mbar_wait(&B.full[0], 0, p.err);
-        if (ok) {
-          dev::tc_fence_after();
-          issue_s(0);
-        }
-      }
-      for (int k = 0; k < ntiles && ok; ++k) {
-        if (k + 1 < ntiles) {
-          ok = dev::mbar_wait(&B.full[(k + 1) % NST], (uint32_t)(((k + 1) / NST) & 1), p.err);
-          if (ok && k + 1 >= 2) ok = dev::mbar_wait(&B.s_free[(k + 1) & 1], (uint32_t)((((k + 1) >> 1) - 1) & 1), p.err);
+      bool ok = true;
+      int g0 = 0, nu = 0;  // first tile of the current unit; units done
+      for (int idx = blockIdx.x; idx < nunits && ok; idx += gridDim.x, ++nu) {
+        const Unit u = unit_of(idx);
+        ok = dev::mbar_wait(B.q_full, (uint32_t)(nu & 1), p.err);  // this unit's Q rows are in place
+        if (ok && u.ntiles > 0) ok = issue_s(g0);
+        if (ok && u.ntiles > 1) ok = issue_s(g0 + 1);
+        for (int k = 0; k < u.ntiles && ok; ++k) {
+          const int g = g0 + k;
+          ok = dev::mbar_wait(B.p_full, (uint32_t)(g & 1), p.err) &&
+               dev::mbar_wait(&B.vfull[g % NSV], (uint32_t)((g / NSV) & 1), p.err);
+          // the previous unit's O has been read out before this unit overwrites it
+          if (ok && k == 0 && nu > 0) ok = dev::mbar_wait(B.o_free, (uint32_t)((nu - 1) & 1), p.err);
           if (!ok) break;
           dev::tc_fence_after();
-          issue_s(k + 1);
-        }
-        ok = dev::mbar_wait(B.p_full, (uint32_t)(k & 1), p.err);
-        if (!ok) break;
-        dev::tc_fence_after();
-        const uint32_t vb = ring_u32 + (uint32_t)((k % NST) * C::STAGE + C::KVT);
+          const uint64_t vb = dv + (uint64_t)(((g % NSV) * C::KVT) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS_O; ++ks) {
-          // A = P (K-major, 16 keys per step); B = V (MN-major: d contiguous,
-          // 64-wide chunks kChunk apart, 8-key row groups 1024 bytes apart)
-          const uint32_t aoff = (uint32_t)((ks >> 2) * kChunk + (ks & 3) * 32);
-          dev::umma_ss(t_o, dev::umma_desc_sw128(p_u32 + aoff, 16, 1024),
-                       dev::umma_desc_sw128(vb + (uint32_t)(ks * 16 * 128), kChunk, 1024), idesc_o,
-                       (k > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < C::KSTEPS_O; ++ks) {
+            // A = P (K-major, 16 keys per step); B = V (MN-major: d contiguous,
+            // 64-wide chunks kChunk apart, 8-key row groups 1024 bytes apart)
+            const uint64_t aoff = (uint64_t)(((ks >> 2) * kChunk + (ks & 3) * 32) >> 4);
+            dev::umma_ss(t_o, dp + aoff, vb + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, (k > 0 || ks > 0) ? 1u : 0u);
+          }
+          dev::umma_commit(B.o_full);
+          dev::umma_commit(&B.vempty[g % NSV]);
+          if (k + 2 < u.ntiles) ok = issue_s(g + 2);
         }
-        dev::umma_commit(B.o_full);
-        dev::umma_commit(&B.empty[k % NST]);
+        g0 += u.ntiles;
       }
       // every MMA issued above has completed before TMEM may be freed
       dev::umma_commit(B.done);
@@ -296,135 +336,167 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ======================= rows: softmax, P, output =========================
-    const int quarter = warp & 3;
+    // Thread = (row r, half hh): keys [64 hh, 64 hh + 64) of each tile and O
+    // columns [hh D/2, (hh+1) D/2).  The two warps of a lane quarter meet at
+    // named barrier 1 + quarter; they run the same units and tiles and pass
+    // the same barriers even after a timed-out wait (then they skip the
+    // remaining waits), so neither can be left waiting.
+    constexpr int HK = kKeys / 2, HD = D / 2;
+    const int quarter = warp & 3, hh = (warp - 2) >> 2;
     const int r = 32 * quarter + lane;  // this thread's row (its TMEM lane)
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
-    const bool valid = r < qn * G;
-    const int pos = pos0 + q0 + r / G;  // the row's position: keys <= pos
-    const int64_t grow = ((int64_t)(first + q0 + r / G) * hq + (int64_t)h * G + r % G) * D;
-    // ---- Q row into the swizzled Q tile (zero for rows past the unit) ----
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + grow * 2);
-#pragma unroll
-      for (int c = 0; c < C::NCH; ++c) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = valid ? __ldg(src + c * 8 + u) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(qs + c * kChunk + swz(r, u)) = v;
-        }
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(B.q_full);
-    }
-    float ref = -1e30f, lsum = 0.f;
+    const int pair_bar = 1 + quarter;
+    float* xmax = reinterpret_cast<float*>(smem + L.xch);  // [tile parity][half][row]
+    float* xsum = xmax + 2 * 2 * 128;                       // [half][row]
     bool ok = true;
-    for (int k = 0; k < ntiles && ok; ++k) {
-      ok = __all_sync(0xffffffffu, dev::mbar_wait(&B.s_full[k & 1], (uint32_t)((k >> 1) & 1), p.err));
-      if (!ok) break;
-      dev::tc_fence_after();
-      float sv[kKeys];
+    auto wait_ok = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(0xffffffffu, dev::mbar_wait(bar, parity, p.err));
+    };
+    int g0 = 0;
+    for (int idx = blockIdx.x; idx < nunits; idx += gridDim.x) {
+      const Unit u = unit_of(idx);
+      const bool valid = r < u.qn * G;
+      const int pos = u.pos0 + u.q0 + r / G;  // the row's position: keys <= pos
+      const int64_t grow = ((int64_t)(u.first + u.q0 + r / G) * hq + (int64_t)u.h * G + r % G) * D;
+      // ---- this half of the Q row into the swizzled Q tile (zero for rows
+      // past the unit); the previous unit's MMAs have all completed (its
+      // output was read after them)
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + grow * 2);
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t w[32];
-        dev::tmem_ld32(t_s0 + (uint32_t)((k & 1) * kKeys + 32 * c) + lane_addr, w);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[32 * c + i] = __uint_as_float(w[i]);
-      }
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&B.s_free[k & 1]);
-      // mask and scale; the row's max over this tile
-      const int key0 = k * kKeys;
-      const int lim = min(pos + 1, seq_len) - key0;  // keys [key0, key0 + lim) are visible
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < kKeys; ++i) {
-        sv[i] = (valid && i < lim) ? sv[i] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sv[i]);
-      }
-      // the previous PV MMA has finished: P may be rewritten, O is stable
-      if (k > 0) {
-        ok = __all_sync(0xffffffffu, dev::mbar_wait(B.o_full, (uint32_t)((k - 1) & 1), p.err));
-        if (!ok) break;
-        dev::tc_fence_after();
-      }
-      const bool move = mx > ref + kRefSlack;
-      const float alpha = move ? dev::ex2(ref - mx) : 1.f;
-      if (k > 0 && __any_sync(0xffffffffu, move)) {
-        // rescale this row of O in TMEM (rows that keep their reference use 1)
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t w[32];
-          const uint32_t ta = t_o + (uint32_t)(32 * c) + lane_addr;
-          dev::tmem_ld32(ta, w);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-          dev::tmem_st32(ta, w);
+        for (int v = hh * C::NCH * 4; v < (hh + 1) * C::NCH * 4; ++v) {
+          const uint4 x = valid ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(qs + (v >> 3) * kChunk + swz(r, v & 7)) = x;
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(B.q_full);
       }
-      if (move) {
-        lsum *= alpha;
-        ref = mx;
-      }
-      // P = 2^(s - ref) as bf16 into the swizzled P tile; the running sum
-      float ps_row = 0.f;
+      float ref = -1e30f, lsum = 0.f;
+      for (int k = 0; k < u.ntiles; ++k) {
+        const int g = g0 + k;
+        wait_ok(&B.s_full[g & 1], (uint32_t)((g >> 1) & 1));
+        dev::tc_fence_after();
+        float sv[HK];
+        {
+          uint32_t w[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < HK / 32; ++c) {
+            dev::tmem_ld32(t_s0 + (uint32_t)((g & 1) * kKeys + HK * hh + 32 * c) + lane_addr, w);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = dev::ex2(sv[64 * c + 8 * u + 2 * e] - ref);
-            const float b = dev::ex2(sv[64 * c + 8 * u + 2 * e + 1] - ref);
-            ps_row += a + b;
-            pk[e] = dev::pack_bf16(a, b);
+            for (int i = 0; i < 32; ++i) sv[32 * c + i] = __uint_as_float(w[i]);
           }
-          *reinterpret_cast<uint4*>(ps + c * kChunk + swz(r, u)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-      }
-      lsum += ps_row;
-      // the tile holding the context's end: slots past it hold stale pool
-      // bytes (masked scores, but 0 * NaN would poison P V): zero their V rows
-      const int stale0 = seq_len - key0, stale1 = min(kKeys, nbneed * BS - key0);
-      if (stale0 < stale1) {
-        uint8_t* vt = ring + (size_t)(k % NST) * C::STAGE + C::KVT;
-        const int units = (stale1 - stale0) * C::NCH * 8;
-        for (int i = tid - 64; i < units; i += 128) {
-          const int key = stale0 + i / (C::NCH * 8), rest = i % (C::NCH * 8);
-          *reinterpret_cast<uint4*>(vt + (rest >> 3) * kChunk + key * 128 + (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
-        }
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(B.p_full);
-    }
-    // ---- O / sum -> output row ----
-    if (ok && ntiles > 0) {
-      ok = __all_sync(0xffffffffu, dev::mbar_wait(B.o_full, (uint32_t)((ntiles - 1) & 1), p.err));
-      if (ok) {
-        dev::tc_fence_after();
-        const float inv = valid ? 1.f / lsum : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + grow * 2);
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t w[32];
-          dev::tmem_ld32(t_o + (uint32_t)(32 * c) + lane_addr, w);
-          if (valid) {
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&B.s_free[g & 1]);
+        // mask; this half's max, then the row's (the scale is positive, so
+        // it is applied to the max and folded into the exponent's FMA)
+        const int lim = min(pos + 1, u.seq_len) - k * kKeys - HK * hh;  // keys [0, lim) of this half are visible
+        float mp[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+        for (int i = 0; i < 4; ++i) mp[i] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < HK; ++i) {
+          sv[i] = (valid && i < lim) ? sv[i] : -INFINITY;
+          mp[i & 3] = fmaxf(mp[i & 3], sv[i]);
+        }
+        const float mh = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        xmax[((g & 1) * 2 + hh) * 128 + r] = mh;
+        dev::named_bar_sync(pair_bar, 64);
+        const float mx = fmaxf(mh, xmax[((g & 1) * 2 + (hh ^ 1)) * 128 + r]) * p.scale_log2;
+        const bool move = mx > ref + kRefSlack;
+        const float alpha = move ? dev::ex2(ref - mx) : 1.f;
+        if (move) {
+          lsum *= alpha;
+          ref = mx;
+        }
+        // P = 2^(s * scale - ref) as bf16 pairs, in registers: this work
+        // overlaps the previous tile's PV MMA
+        uint32_t pk[HK / 2];
+        float sp[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sp[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < HK / 2; ++i) {
+          const float a = dev::ex2(fmaf(sv[2 * i], p.scale_log2, -ref));
+          const float b = dev::ex2(fmaf(sv[2 * i + 1], p.scale_log2, -ref));
+          sp[i & 3] += a + b;
+          pk[i] = dev::pack_bf16(a, b);
+        }
+        lsum += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+        // the previous PV MMA has finished: P may be rewritten, O is stable
+        if (k > 0) {
+          wait_ok(B.o_full, (uint32_t)((g - 1) & 1));
+          dev::tc_fence_after();
+          if (__any_sync(0xffffffffu, move)) {
+            // rescale this row's half of O in TMEM (rows that keep their
+            // reference use 1)
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
+              uint32_t w[32];
+              const uint32_t ta = t_o + (uint32_t)(HD * hh + 32 * c) + lane_addr;
+              dev::tmem_ld32(ta, w);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+              dev::tmem_st32(ta, w);
+            }
+          }
+        }
+        // this half's 64 keys are chunk hh of the swizzled P tile
+#pragma unroll
+        for (int uu = 0; uu < 8; ++uu)
+          *reinterpret_cast<uint4*>(ps + hh * kChunk + swz(r, uu)) =
+              make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+        // the tile holding the context's end: slots past it hold stale pool
+        // bytes (masked scores, but 0 * NaN would poison P V): zero their V rows
+        const int key0 = k * kKeys;
+        const int stale0 = u.seq_len - key0, stale1 = min(kKeys, u.nbneed * BS - key0);
+        if (stale0 < stale1) {
+          wait_ok(&B.vfull[g % NSV], (uint32_t)((g / NSV) & 1));
+          uint8_t* vt = vring + (size_t)(g % NSV) * C::KVT;
+          const int units = (stale1 - stale0) * C::NCH * 8;
+          for (int i = tid - 64; i < units; i += 32 * kRowWarps) {
+            const int key = stale0 + i / (C::NCH * 8), rest = i % (C::NCH * 8);
+            *reinterpret_cast<uint4*>(vt + (rest >> 3) * kChunk + key * 128 + (rest & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(B.p_full);
+      }
+      // ---- O / sum -> this half of the output row; then O is free ----
+      if (u.ntiles > 0) {
+        wait_ok(B.o_full, (uint32_t)((g0 + u.ntiles - 1) & 1));
+        dev::tc_fence_after();
+        xsum[hh * 128 + r] = lsum;
+        dev::named_bar_sync(pair_bar, 64);
+        const float total = lsum + xsum[(hh ^ 1) * 128 + r];
+        const float inv = valid ? 1.f / total : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (grow + HD * hh) * 2);
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t w[32];
+          dev::tmem_ld32(t_o + (uint32_t)(HD * hh + 32 * c) + lane_addr, w);
+          if (valid && ok) {
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                pk[e] = dev::pack_bf16(__uint_as_float(w[8 * u + 2 * e]) * inv,
-                                       __uint_as_float(w[8 * u + 2 * e + 1]) * inv);
-              dst[4 * c + u] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                pk[e] = dev::pack_bf16(__uint_as_float(w[8 * uu + 2 * e]) * inv,
+                                       __uint_as_float(w[8 * uu + 2 * e + 1]) * inv);
+              dst[4 * c + uu] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           }
         }
       }
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(B.o_free);
+      g0 += u.ntiles;
     }
   }
 
@@ -441,7 +513,7 @@ template <int D, int BS>
 cudaError_t launch_u(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v, int grid,
                      cudaStream_t stream) {
   using C = U<D, BS>;
-  const ULayout L = u_layout(C::QBYTES, C::STAGE, p.nstages, p.rows.num_seqs);
+  const ULayout L = u_layout(C::QBYTES, C::KVT, p.nstages, p.nstages_v, p.rows.num_seqs);
   auto kern = prefill_umma_kernel<D, BS>;
   static int set_for[64] = {0};
   int dev = 0;
@@ -473,19 +545,20 @@ bool prefill_umma_supported(int kv, int q, int head_dim, int block_size, int gro
 }
 
 cudaError_t launch_prefill_umma(const PrefillParams& p_in, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                int head_dim, int block_size, int num_tokens, cudaStream_t stream) {
+                                int head_dim, int block_size, int num_tokens, int num_sms, cudaStream_t stream) {
   PrefillParams p = p_in;
   const int nch = head_dim / 64;
-  const int qbytes = nch * kChunk, stage = 2 * nch * kChunk;
-  const int fixed = (int)u_layout(qbytes, stage, 0, p.rows.num_seqs).total;
-  int nst = (kSmemOptIn - fixed) / (stage + 16);
-  if (nst > 4) nst = 4;
-  if (nst < 2) return cudaErrorNotSupported;  // too many sequences for the unit table: caller falls back
-  p.nstages = nst;
+  const int qbytes = nch * kChunk, kvt = nch * kChunk;
+  const int fixed = (int)u_layout(qbytes, kvt, 0, 0, p.rows.num_seqs).total;
+  const int nbuf = (kSmemOptIn - fixed) / (kvt + 16);  // K and V stages that fit
+  const int nsk = min(4, nbuf / 2), nsv = min(4, nbuf - nbuf / 2);
+  if (nsk < 2 || nsv < 2) return cudaErrorNotSupported;  // too many sequences for the unit table: caller falls back
+  p.nstages = nsk;
+  p.nstages_v = nsv;
   const int qb = kRows / p.group;
-  const int64_t grid = ((int64_t)num_tokens / qb + p.rows.num_seqs) * p.num_kv_heads;
-  if (grid <= 0) return cudaSuccess;
-  if (grid > INT32_MAX) return cudaErrorNotSupported;
+  const int64_t bound = ((int64_t)num_tokens / qb + p.rows.num_seqs) * p.num_kv_heads;  // units, at most
+  if (bound <= 0) return cudaSuccess;
+  const int64_t grid = bound < num_sms ? bound : num_sms;  // one persistent CTA per SM
   if (head_dim == 128 && block_size == 16) return launch_u<128, 16>(p, tm_k, tm_v, (int)grid, stream);
   if (head_dim == 128 && block_size == 32) return launch_u<128, 32>(p, tm_k, tm_v, (int)grid, stream);
   if (head_dim == 64 && block_size == 16) return launch_u<64, 16>(p, tm_k, tm_v, (int)grid, stream);

@@ -147,6 +147,9 @@ MIXED_EDGE = {
     "group3_prefill": dict(context_lens=[4, 0], q_lens=[9, 22], num_q_heads=6, num_kv_heads=2),  # CUDA cores
     "prefill_only": dict(context_lens=[0, 200], q_lens=[33, 100]),
     "fp8_prefill": dict(context_lens=[0, 40], q_lens=[17, 30], kv_dtype="e4m3"),  # CUDA cores
+    # more prompt units than SMs: persistent CTAs chain several units
+    "many_units": dict(context_lens=[7 * i for i in range(40)] + [5, 9], q_lens=[40] * 40 + [1, 1],
+                       num_q_heads=8, num_kv_heads=2),
 }
 
 
