@@ -163,7 +163,13 @@ size_t pa_prefill_workspace_size(const pa_cache_desc* desc, int32_t num_seqs, in
  *                   non-decreasing, query_start_loc[num_seqs] = num_tokens
  *   seq_lens        device, int32 [num_seqs], seq_lens[s] >= q_len_s
  *   max_q_len       host, >= every q_len_s
- *   workspace       as for pa_decode, sized by pa_prefill_workspace_size. */
+ *   workspace       as for pa_decode, sized by pa_prefill_workspace_size.
+ * Decode rows (q_len_s = 1) run on pa_decode's kernels.  Prompt rows of a
+ * bf16 pool with bf16 queries run on a tcgen05 kernel (TMEM accumulators)
+ * when the GQA group divides 128 and the batch's unit table fits in shared
+ * memory, else on an mma.sync kernel when the group divides 64, else on the
+ * CUDA-core kernel; every dtype and group is served.  Errors and the
+ * workspace error word are as for pa_decode. */
 int pa_decode_chunked_prefill(const pa_cache_desc* desc, const void* q, const void* k_cache,
                               const void* v_cache, const int32_t* block_tables,
                               int32_t max_blocks_per_seq, const int32_t* query_start_loc,

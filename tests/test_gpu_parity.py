@@ -143,6 +143,9 @@ MIXED_EDGE = {
     "mha_prefill": dict(context_lens=[3, 70, 0], q_lens=[64, 65, 130], num_q_heads=2, num_kv_heads=2),
     "group8_prefill": dict(context_lens=[0, 21, 9], q_lens=[8, 9, 40], num_q_heads=16, num_kv_heads=2),
     "group16_prefill": dict(context_lens=[0, 33], q_lens=[5, 37], num_q_heads=32, num_kv_heads=2),
+    "group32_prefill": dict(context_lens=[0, 20, 100], q_lens=[9, 30, 1], num_q_heads=64, num_kv_heads=2),
+    "head64_many_units": dict(context_lens=[3 * i for i in range(30)], q_lens=[70] * 30, num_q_heads=8,
+                              num_kv_heads=2, head_dim=64),
     "head64_bs32_prefill": dict(context_lens=[0, 50, 7], q_lens=[70, 3, 1], head_dim=64, block_size=32),
     "group3_prefill": dict(context_lens=[4, 0], q_lens=[9, 22], num_q_heads=6, num_kv_heads=2),  # CUDA cores
     "prefill_only": dict(context_lens=[0, 200], q_lens=[33, 100]),
