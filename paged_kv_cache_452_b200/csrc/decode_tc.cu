@@ -151,9 +151,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  // Everything read below may have been produced by the previous kernel in
-  // the stream (programmatic dependent launch lets this grid start early).
-  dev::grid_dep_wait();
+  // Programmatic dependent launch lets this grid start while the previous
+  // kernel in the stream (normally the step's cache write) still runs.  The
+  // prologue below reads only the step's inputs (lengths, query offsets,
+  // block tables) and this call's workspace, which no kernel of the step
+  // writes; the K/V pool and the queries are touched only after the wait
+  // placed before the first copy is issued.
 
   // ---- blocks per sequence, exclusive prefix over the batch ----------------
   for (int s = tid; s < S; s += kThreads) {
@@ -294,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
     }
   };
   int issued = 0;
+  dev::grid_dep_wait();  // the pool rows this step wrote are visible from here on
   for (; issued < NSW && issued < nmine; ++issued) issue(issued);
   nxt = describe(32);  // the next batch, needed from warp-tile 32 on
 
