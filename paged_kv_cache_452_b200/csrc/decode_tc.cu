@@ -587,43 +587,41 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSM)
       }
       ready = __shfl_sync(0xffffffffu, ready, 0);
       __syncwarp();
-      // running max per query column over this warp and every contributor
-      float M0 = m0, M1 = m1;
-      for (int c = cf + 1; c <= cl && ready; ++c) {
-        if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
-        const float* pml = p.ws.ml + (int64_t)c * G * 2;
-        if (c0 < G) M0 = fmaxf(M0, __ldcg(pml + c0 * 2));
-        if (c1 < G) M1 = fmaxf(M1, __ldcg(pml + c1 * 2));
-      }
-      const float e0 = dev::ex2(m0 - M0), e1 = dev::ex2(m1 - M1);
-      float L0 = l0 * e0, L1 = l1 * e1;
-#pragma unroll
-      for (int mt = 0; mt < C::DM; ++mt) {
-        o[mt][0] *= e0;
-        o[mt][2] *= e0;
-        o[mt][1] *= e1;
-        o[mt][3] *= e1;
-      }
+      // fold each contributor into this warp's state with a running
+      // log-sum-exp: its (max, sum) and its outputs are loaded together, so
+      // a contributor costs one round trip to L2
+      float M0 = m0, M1 = m1, L0 = l0, L1 = l1;
       for (int c = cf + 1; c <= cl && ready; ++c) {
         if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
         const float* pml = p.ws.ml + (int64_t)c * G * 2;
         const float* po = p.ws.o + (int64_t)c * G * D;
-        const float w0 = c0 < G ? dev::ex2(__ldcg(pml + c0 * 2) - M0) : 0.f;
-        const float w1 = c1 < G ? dev::ex2(__ldcg(pml + c1 * 2) - M1) : 0.f;
-        if (c0 < G) L0 += __ldcg(pml + c0 * 2 + 1) * w0;
-        if (c1 < G) L1 += __ldcg(pml + c1 * 2 + 1) * w1;
+        const float mc0 = c0 < G ? __ldcg(pml + c0 * 2) : -INFINITY;
+        const float mc1 = c1 < G ? __ldcg(pml + c1 * 2) : -INFINITY;
+        const float lc0 = c0 < G ? __ldcg(pml + c0 * 2 + 1) : 0.f;
+        const float lc1 = c1 < G ? __ldcg(pml + c1 * 2 + 1) : 0.f;
+        float oc[C::DM][4];
 #pragma unroll
         for (int mt = 0; mt < C::DM; ++mt) {
           const int d0 = 16 * mt + g;
-          if (c0 < G) {
-            o[mt][0] += w0 * __ldcg(po + c0 * D + d0);
-            o[mt][2] += w0 * __ldcg(po + c0 * D + d0 + 8);
-          }
-          if (c1 < G) {
-            o[mt][1] += w1 * __ldcg(po + c1 * D + d0);
-            o[mt][3] += w1 * __ldcg(po + c1 * D + d0 + 8);
-          }
+          oc[mt][0] = c0 < G ? __ldcg(po + c0 * D + d0) : 0.f;
+          oc[mt][2] = c0 < G ? __ldcg(po + c0 * D + d0 + 8) : 0.f;
+          oc[mt][1] = c1 < G ? __ldcg(po + c1 * D + d0) : 0.f;
+          oc[mt][3] = c1 < G ? __ldcg(po + c1 * D + d0 + 8) : 0.f;
         }
+        const float n0 = fmaxf(M0, mc0), n1 = fmaxf(M1, mc1);
+        const float a0 = dev::ex2(M0 - n0), a1 = dev::ex2(M1 - n1);
+        const float w0 = dev::ex2(mc0 - n0), w1 = dev::ex2(mc1 - n1);
+        L0 = L0 * a0 + lc0 * w0;
+        L1 = L1 * a1 + lc1 * w1;
+#pragma unroll
+        for (int mt = 0; mt < C::DM; ++mt) {
+          o[mt][0] = o[mt][0] * a0 + oc[mt][0] * w0;
+          o[mt][2] = o[mt][2] * a0 + oc[mt][2] * w0;
+          o[mt][1] = o[mt][1] * a1 + oc[mt][1] * w1;
+          o[mt][3] = o[mt][3] * a1 + oc[mt][3] * w1;
+        }
+        M0 = n0;
+        M1 = n1;
       }
       // L0/L1 are whole-column sums already: l0/l1 were reduced over the
       // warp above and a partial's sum is per column
