@@ -60,8 +60,7 @@ struct DecodeParams {
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                              int kv, int head_dim, int block_size, int num_sms, cudaStream_t stream);
 size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages);
-int decode_tc_workers(int num_sms);
-int decode_tc_grid(int num_sms);
+int decode_tc_workers(int num_sms);  // the most worker warps a launch can have (workspace sizing)
 size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms);
 
 // Prompt rows (q_len > 1) of a mixed step on the tensor-core path.
