@@ -161,6 +161,17 @@ def test_mixed_edge_cases(case, cuda_device):
     run_and_check(W.custom(case, **MIXED_EDGE[case]), cuda_device)
 
 
+def test_mixed_step_with_more_sequences_than_the_unit_table_holds(cuda_device):
+    """8 502 sequences: the tcgen05 prefill kernel's per-sequence unit table no
+    longer fits next to two K and two V stages, so the prompt rows fall back
+    to the mma.sync prefill kernel (and the decode rows run at two CTAs per
+    SM); the result must not change."""
+    n = 8500
+    wl = W.custom("many_sequences_mixed", context_lens=[5 + (i % 11) for i in range(n)] + [10, 40],
+                  q_lens=[1] * n + [20, 33], num_q_heads=8, num_kv_heads=2)
+    run_and_check(wl, cuda_device, seqs=[0, 1, 7, 4999, n - 1, n, n + 1])
+
+
 def test_paged_output_equals_contiguous_output(cuda_device):
     """Paging changes nothing: the same draws through a shuffled free list and
     through an identity free list (contiguous blocks) give bit-identical
