@@ -8,6 +8,7 @@ Contents
 --------
 * ``cache_write`` / ``attention`` / ``e4m3_decode`` / ``e4m3_encode``: numpy
   front ends of the fp64 C oracle in ``pa_oracle.c`` (built with gcc).
+* ``copy_blocks``: whole-block copies inside the pools (copy-on-write).
 * ``pool_model.BlockPoolModel``: a dict/list restatement of the block pool
   (free_block_queue, ref_cnt, hash-keyed prefix sharing).
 * ``admission``: the pages' memory arithmetic (blocks per sequence, bytes per
@@ -122,6 +123,17 @@ def cache_write(k_new, v_new, slot_mapping, k_cache, v_cache, in_dtype, kv_dtype
                                   float(k_scale), float(v_scale), _ptr(k_cache), _ptr(v_cache))
     if rc != 0:
         raise ValueError("slot past the end of the pool")
+
+
+def copy_blocks(k_cache, v_cache, pairs):
+    """Copy-on-write's device half ("PagedAttention：KV cache 即虚拟内存
+    (block manager & 碎片)", 深入原理, 共享 → prefix caching: a fork that
+    diverges inside a shared block triggers a copy): for each (src, dst)
+    pair, block dst of each pool becomes block src, every kv head and slot
+    in the storage format.  In place."""
+    for src, dst in pairs:
+        k_cache[dst] = k_cache[src]
+        v_cache[dst] = v_cache[src]
 
 
 def attention(q, row_seq, row_pos, block_tables, k_cache, v_cache, kv_dtype, num_q_heads,

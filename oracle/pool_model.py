@@ -21,7 +21,11 @@ Follows
   - 共享 → prefix caching: a block is keyed by the hash of its tokens and
     its parent's hash; equal prefixes give equal hashes, so a second request
     points at the existing block and ``touch()`` raises its ``ref_cnt``;
-    only whole blocks are shared.
+    only whole blocks are shared; a fork that diverges inside a shared block
+    triggers copy-on-write.
+* "49 vLLM / PagedAttention", Почему это важно and, under Вопросы пытливого
+  ума, the prefix-sharing answer: blocks shared between requests are
+  copy-on-write, like pages shared between processes.
 
 Readings where the pages are silent
 -----------------------------------
@@ -38,6 +42,17 @@ Readings where the pages are silent
   tail of a sequence is evicted before its (possibly shared) prefix.
 * Allocation is all-or-nothing: on shortage nothing changes.
 * ``append`` takes no token ids, so blocks filled by decoding are never hashed.
+* Fork (copy-on-write): ``fork(parent, child)`` gives the child the parent's
+  length and block table and raises every block's ``ref_cnt`` by one.  When
+  ``append`` is about to write into a sequence's last block while that block
+  is partly filled and shared (``ref_cnt`` > 1), the sequence first moves to
+  a new block popped from the head: the pair (shared block, new block) is
+  queued for the caller to copy on the device, the shared block's
+  ``ref_cnt`` drops by one, and the new block (never hashed) replaces it in
+  the table.  A full shared block is never copied: the next token opens a
+  new block anyway.  The copy's block counts toward the all-or-nothing
+  check.  ``take_copies`` returns the queued pairs, oldest first, and
+  empties the queue.
 """
 from collections import OrderedDict
 
@@ -79,6 +94,7 @@ class BlockPoolModel:
         self.block_key = [None] * num_blocks  # (hash, tokens) while cached
         self.hash_to_block = {}
         self.seqs = {}  # seq_id -> {"blocks": [...], "num_tokens": n}
+        self.copies = []  # (src, dst) block pairs queued by copy-on-write
 
     # -- queries -------------------------------------------------------------
     def num_free(self):
@@ -163,9 +179,16 @@ class BlockPoolModel:
         bs = self.block_size
         blocks = seq["blocks"]
         start = seq["num_tokens"]
-        need = max(0, (start + n_new + bs - 1) // bs - len(blocks))
+        cow = n_new > 0 and start % bs != 0 and self.ref_cnt[blocks[-1]] > 1
+        need = max(0, (start + n_new + bs - 1) // bs - len(blocks)) + (1 if cow else 0)
         if need > len(self.free_queue):
             raise PoolModelError("NO_BLOCKS", f"need {need} blocks")
+        if cow:  # the shared, partly filled last block: copy it first
+            src = blocks[-1]
+            dst = self._pop_head()
+            self.ref_cnt[src] -= 1
+            blocks[-1] = dst
+            self.copies.append((src, dst))
         slots = []
         for p in range(start, start + n_new):
             if len(blocks) * bs <= p:  # the block-table snippet's test
@@ -173,6 +196,20 @@ class BlockPoolModel:
             slots.append(blocks[p // bs] * bs + p % bs)
         seq["num_tokens"] = start + n_new
         return slots
+
+    def fork(self, parent_id, child_id):
+        """A new sequence with the parent's length and blocks, all shared."""
+        parent = self._seq(parent_id)
+        if child_id in self.seqs:
+            raise PoolModelError("INVALID_ARG", f"sequence {child_id} exists")
+        for b in parent["blocks"]:
+            self.ref_cnt[b] += 1
+        self.seqs[child_id] = {"blocks": list(parent["blocks"]), "num_tokens": parent["num_tokens"]}
+
+    def take_copies(self):
+        """The (src, dst) pairs queued by copy-on-write, oldest first."""
+        out, self.copies = self.copies, []
+        return out
 
     def slots(self, seq_id, start, n):
         """Flat slots of positions [start, start + n) of a sequence."""

@@ -105,6 +105,48 @@ def test_cache_write_index_by_hand():
         oracle.cache_write(k[:1], v[:1], np.array([12]), kc, vc, "f32", "f32")
 
 
+def test_copy_blocks_by_hand():
+    """Block 1 copied to block 3 (and block 0 to block 2), checked element by
+    element against the values written by hand; the other blocks keep theirs."""
+    nb, hkv, bs, d = 4, 2, 4, 3
+    kc, vc = oracle.new_caches(nb, hkv, bs, d, "e4m3")  # V d-major, sentinel 0x7F
+    for b in range(nb):
+        for h in range(hkv):
+            for o in range(bs):
+                for e in range(d):
+                    kc[b, h, o, e] = (b * 64 + h * 16 + o * 4 + e) % 127
+                    vc[b, h, e, o] = (b * 32 + h * 8 + e * 4 + o + 1) % 127
+    k0, v0 = kc.copy(), vc.copy()
+    oracle.copy_blocks(kc, vc, [(1, 3), (0, 2)])
+    for h in range(hkv):
+        for o in range(bs):
+            for e in range(d):
+                assert kc[3, h, o, e] == (64 + h * 16 + o * 4 + e) % 127
+                assert vc[3, h, e, o] == (32 + h * 8 + e * 4 + o + 1) % 127
+                assert kc[2, h, o, e] == (h * 16 + o * 4 + e) % 127
+                assert vc[2, h, e, o] == (h * 8 + e * 4 + o + 1) % 127
+    assert np.array_equal(kc[:2], k0[:2]) and np.array_equal(vc[:2], v0[:2])
+    oracle.copy_blocks(kc, vc, [])
+    assert np.array_equal(kc[:2], k0[:2])
+
+
+def test_copy_blocks_keeps_attention():
+    """A table that points at the copy gives the same fp64 output as one that
+    points at the original (what copy-on-write relies on)."""
+    p = _paged_problem([40], 4, 2, 16, 16, seed=3, shuffle=True)
+    kc, vc, tab = p["kc"], p["vc"], p["tables"]
+    used = set(tab[0][tab[0] >= 0].tolist())
+    free = [b for b in range(kc.shape[0]) if b not in used][:1]
+    src = int(tab[0, 1])
+    oracle.copy_blocks(kc, vc, [(src, free[0])])
+    moved = tab.copy()
+    moved[0, 1] = free[0]
+    q = np.random.default_rng(4).standard_normal((1, 4, 16))
+    oa = oracle.attention(q, [0], [39], tab, kc, vc, "f32", 4, 0.25)
+    ob = oracle.attention(q, [0], [39], moved, kc, vc, "f32", 4, 0.25)
+    assert np.array_equal(oa, ob)
+
+
 def test_cache_write_bf16_is_bit_copy():
     nb, hkv, bs, d = 4, 2, 16, 8
     kc = oracle.new_cache(nb, hkv, bs, d, "bf16")

@@ -138,3 +138,59 @@ def test_hash_depends_on_parent_and_tokens():
     assert fnv1a64(b"foobar") == 0x85944171F73967E8
     # parent (8 bytes LE) then int32 LE token ids
     assert block_hash(5, [1]) == fnv1a64(bytes([5, 0, 0, 0, 0, 0, 0, 0, 1, 0, 0, 0]))
+
+
+def test_fork_shares_blocks_and_copies_on_write_when_a_sequence_diverges():
+    # hand-derived trace, block size 4, free queue 6 2 5 0 7 1 3 4
+    pool = BlockPoolModel(8, 4, initial_free_order=[6, 2, 5, 0, 7, 1, 3, 4])
+    pool.add_seq("p", 6)  # positions 0..3 in block 6, 4..5 in block 2 (half full)
+    pool.fork("p", "c")
+    assert pool.block_table("c") == [6, 2] and pool.num_tokens("c") == 6
+    assert pool.ref_cnt[6] == 2 and pool.ref_cnt[2] == 2
+    assert pool.take_copies() == []
+    # the child writes position 6 into the shared, half-full block 2: it
+    # moves to a copy in block 5 (head of the queue) and writes slot 5*4+2
+    assert pool.append("c", 1) == [22]
+    assert pool.block_table("c") == [6, 5] and pool.block_table("p") == [6, 2]
+    assert (pool.ref_cnt[2], pool.ref_cnt[5], pool.ref_cnt[6]) == (1, 1, 2)
+    assert pool.take_copies() == [(2, 5)]
+    assert pool.take_copies() == []  # taken once
+    # the parent is now block 2's only owner: it writes in place
+    assert pool.append("p", 2) == [10, 11]
+    assert pool.take_copies() == []
+    # a full shared block is never copied: the next token opens block 0
+    pool.fork("p", "d")
+    assert pool.append("d", 1) == [0]
+    assert pool.block_table("d") == [6, 2, 0] and pool.take_copies() == []
+    assert (pool.ref_cnt[6], pool.ref_cnt[2]) == (3, 2)
+    # release walks blocks in reverse: c's block 5 goes to the tail, 6 stays
+    pool.free_seq("c")
+    assert pool.free_order() == [7, 1, 3, 4, 5] and pool.ref_cnt[6] == 2
+
+
+def test_copy_on_write_is_all_or_nothing():
+    pool = BlockPoolModel(2, 4)
+    pool.add_seq("a", 5)  # blocks 0 (full) and 1 (one token)
+    pool.fork("a", "b")
+    with pytest.raises(PoolModelError) as e:
+        pool.append("b", 1)  # the copy needs a block and none is free
+    assert e.value.code == "NO_BLOCKS"
+    assert pool.block_table("b") == [0, 1] and pool.ref_cnt == [2, 2]
+    assert pool.num_tokens("b") == 5 and pool.take_copies() == []
+    with pytest.raises(PoolModelError):
+        pool.fork("a", "b")  # the child exists
+    with pytest.raises(PoolModelError):
+        pool.fork("zz", "e")  # no such parent
+    pool.append("b", 0)  # nothing to write: no copy, no block
+    assert pool.take_copies() == []
+
+
+def test_fork_of_an_empty_sequence_and_release_of_both():
+    pool = BlockPoolModel(3, 4)
+    pool.add_seq("a", 0)
+    pool.fork("a", "b")
+    assert pool.block_table("b") == [] and pool.append("b", 2) == [0, 1]
+    assert pool.take_copies() == []  # no shared block to copy
+    pool.free_seq("a")
+    pool.free_seq("b")
+    assert pool.free_order() == [1, 2, 0] and pool.ref_cnt == [0, 0, 0]
