@@ -3,6 +3,9 @@ step's new K/V + pa_decode) on a seeded synthetic batch, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+`--workload block_copy` measures copy-on-write's block copy (pa_copy_blocks)
+instead, as "block copy GB/s" (bytes read + written per step / step time).
+
 Prints one JSON line (rank 0).  `value` is KV GB/s: the step's algorithmic
 attention bytes (every valid token's K and V once, shared prefix blocks
 once, plus queries, outputs, table entries and lengths) divided by the step
@@ -28,13 +31,17 @@ import pa_workloads as W  # noqa: E402
 METRIC = "paged decode attention KV GB/s"
 DEFAULT_WORKLOAD = "gqa_bf16"
 
-# DRAM bytes (read + write) per launch of the decode kernel from one ncu
-# capture (profiles/decode_tc_gqa_bf16.md), valid only for the kernel source
-# that was profiled: any edit to the source drops the figure to null.
+# DRAM bytes (read + write) per launch of the workload's dominant kernel from
+# one ncu capture (profiles/), valid only for the kernel source that was
+# profiled: any edit to the source drops the figure to null.
 PROFILED_TRAFFIC = {
     "gqa_bf16": {"source": "paged_kv_cache_452_b200/csrc/decode_tc.cu",
                  "sha256": "4917a915d6a1f701d21ea655453b162430606a896c07a58cbffe723578f8d162",
                  "bytes": 294_643_200},
+    # profiles/copy_blocks_block_copy.md: mean of two launches
+    "block_copy": {"source": "paged_kv_cache_452_b200/csrc/block_copy.cu",
+                   "sha256": "14c4d4e16d7a6cfba5f9139645ec9d67aba270f8986a597db740b32a1a2c0f11",
+                   "bytes": 488_925_056},
 }
 
 
@@ -401,19 +408,174 @@ def bench_ours(args):
         torch.distributed.destroy_process_group()
 
 
+# Copy-on-write's device half (pa_copy_blocks), measured on its own: random
+# pairs of blocks in the geometry of gqa_bf16's pool (8 kv heads, head_dim
+# 128, 16 slots, bf16: 32 KiB per block per pool).
+BLOCK_COPY = {"pairs": 4096, "num_kv_heads": 8, "head_dim": 128, "block_size": 16}
+BLOCK_COPY_METRIC = "block copy GB/s"
+
+
+def block_copy_geometry():
+    c = BLOCK_COPY
+    block_bytes = c["num_kv_heads"] * c["block_size"] * c["head_dim"] * 2
+    # per step every pair reads and writes one block of each pool
+    return c["pairs"], block_bytes, 2 * 2 * c["pairs"] * block_bytes
+
+
+def block_copy_cpu(budget_s):
+    """The oracle's copy (numpy, one host core) on a bounded sample of pairs."""
+    import oracle
+    n, block_bytes, _ = block_copy_geometry()
+    c = BLOCK_COPY
+    m = max(16, min(1024, n))  # 128 MiB of host blocks; passes repeat until budget_s
+    shape = (2 * m, c["num_kv_heads"], c["block_size"], c["head_dim"])
+    g = np.random.default_rng(0)
+    k = g.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+    v = g.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+    perm = g.permutation(2 * m)
+    pairs = list(zip(perm[:m].tolist(), perm[m:].tolist()))
+    oracle.copy_blocks(k, v, pairs)  # warm
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.copy_blocks(k, v, pairs)
+        reps += 1
+        t = time.perf_counter() - t0
+        if t >= budget_s:
+            break
+    bytes_ = reps * 2 * 2 * m * block_bytes
+    return {"value": bytes_ / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{m} of {n} pairs per pass, {reps} passes, numpy block copies, {t:.2f} s"}
+
+
+def bench_block_copy(args):
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        if rank == 0:
+            per_step = max(0.05, min(args.ref_budget, 150.0 / (args.steps + args.warmup)))
+            base = block_copy_cpu(per_step)
+            line = {"impl": "reference", "metric": BLOCK_COPY_METRIC, "value": base["value"], "unit": "GB/s",
+                    "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                    "config": {"workload": "block_copy", **BLOCK_COPY}, "cpu_baseline": base,
+                    "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import paged_kv_cache_452_b200 as pa
+
+    n, block_bytes, alg_bytes = block_copy_geometry()
+    c = BLOCK_COPY
+    nb = 4 * n  # two pair sets, used alternately: 4 x 256 MiB of blocks per pool set
+    desc = pa.CacheDesc.make(nb, c["block_size"], c["num_kv_heads"], c["num_kv_heads"], c["head_dim"],
+                             "bf16", "bf16")
+    k, v = pa.alloc_cache(desc, device)
+    gen = torch.Generator(device=device).manual_seed(0)
+    for t in (k, v):
+        t.normal_(generator=gen)
+    perm = np.random.default_rng(0).permutation(nb).astype(np.int32)
+    src = [torch.from_numpy(perm[2 * j * n:(2 * j + 1) * n].copy()).to(device) for j in range(2)]
+    dst = [torch.from_numpy(perm[(2 * j + 1) * n:(2 * j + 2) * n].copy()).to(device) for j in range(2)]
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        pa.pa_copy_blocks(desc, src[i & 1], dst[i & 1], k, v)
+    torch.cuda.synchronize()
+    # parity spot check: each destination block equals its source
+    for j in range(2):
+        assert torch.equal(k[dst[j][:64].long()], k[src[j][:64].long()])
+    graphs = []
+    for j in range(2):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            pa.pa_copy_blocks(desc, src[j], dst[j], k, v)
+        graphs.append(gr)
+    for i in range(args.warmup):
+        graphs[i & 1].replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.2 if sampler else 0)
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = _time(lambda i: graphs[i & 1].replay(), args.steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = reduce_max(ms, world, device)
+    clocks = sampler.stop() if sampler else None
+    # end to end through the public API: the pair lists come from pinned host
+    # memory each step and one copied K block goes back to the host
+    src_h = [s_.cpu().pin_memory() for s_ in src]
+    dst_h = [d_.cpu().pin_memory() for d_ in dst]
+    src_d = [torch.empty_like(s_) for s_ in src]
+    dst_d = [torch.empty_like(d_) for d_ in dst]
+    back = torch.empty(k[0].shape, dtype=k.dtype).pin_memory()
+    h2d = 2 * n * 4
+    d2h = back.numel() * back.element_size()
+
+    def e2e_step(i):
+        j = i & 1
+        src_d[j].copy_(src_h[j], non_blocking=True)
+        dst_d[j].copy_(dst_h[j], non_blocking=True)
+        pa.pa_copy_blocks(desc, src_d[j], dst_d[j], k, v)
+        back.copy_(k[int(perm[(2 * j + 1) * n])], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = reduce_max(_time(e2e_step, args.steps, stream), world, device)
+    for gr in graphs:
+        del gr
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    peaks, psrc = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": BLOCK_COPY_METRIC, "value": job_throughput(world, alg_bytes, ms), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "block_copy", **BLOCK_COPY, "block_bytes_per_pool": block_bytes,
+                   "algorithmic_bytes": alg_bytes, "parallelism": f"replicas x{world}",
+                   "step": "pa_copy_blocks over all pairs, replayed as a CUDA graph",
+                   "l2": "two disjoint pair sets used alternately, 256 MiB read per step (> L2)"},
+        "roofline": {"bound": "hbm", "kernel": "copy_blocks_kernel (pa_copy_blocks)", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_source": psrc,
+                     "traffic": profiled_traffic("block_copy"), "kernel_ms": ms},
+        "e2e": {"value": job_throughput(world, alg_bytes, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = block_copy_cpu(min(args.ref_budget, 10.0))
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS) + ["block_copy"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.workload == "block_copy":
+        bench_block_copy(args)
+    elif args.impl == "reference":
         bench_reference(args)
     else:
         bench_ours(args)

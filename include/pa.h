@@ -100,6 +100,21 @@ int pa_cache_write(const pa_cache_desc* desc, const void* k_new, const void* v_n
                    const int64_t* slot_mapping, int32_t num_tokens, void* k_cache, void* v_cache,
                    void* stream);
 
+/* pa_copy_blocks: the device half of copy-on-write ("PagedAttention：KV
+ * cache 即虚拟内存（block manager & 碎片）", 深入原理, 共享 → prefix caching: a
+ * fork that diverges inside a shared block triggers a copy).  For i < n, K
+ * block dst[i] and V block dst[i] become byte copies of blocks src[i]
+ * (every kv head and slot, in the pool's storage format).
+ *   src, dst   device, int32 [n] block ids (from pa_pool_take_copies); a
+ *              pair with an id outside [0, num_blocks), or src == dst, is
+ *              skipped
+ *   k_cache, v_cache  device pools as for pa_cache_write, 16-byte aligned
+ * The pairs run concurrently: no block may be a destination twice, or both
+ * a destination and a source, in one call.  Asynchronous on `stream`; run
+ * it before the pa_cache_write that writes into the new blocks. */
+int pa_copy_blocks(const pa_cache_desc* desc, const int32_t* src, const int32_t* dst, int32_t n,
+                   void* k_cache, void* v_cache, void* stream);
+
 /* Scratch bytes pa_decode needs for num_seqs sequences on the current device. */
 size_t pa_decode_workspace_size(const pa_cache_desc* desc, int32_t num_seqs);
 
@@ -198,7 +213,10 @@ int pa_decode_chunked_prefill(const pa_cache_desc* desc, const void* q, const vo
  *    still be shared (touch() unlinks it); popping it for reuse evicts it;
  *  - release walks a sequence's blocks in reverse logical order;
  *  - every allocation is all-or-nothing (PA_ERR_NO_BLOCKS changes nothing);
- *  - blocks filled by pa_pool_append are never hashed. */
+ *  - blocks filled by pa_pool_append are never hashed;
+ *  - copy-on-write ("分叉触发 copy-on-write" in the same bullet) copies a
+ *    shared block only when a sequence writes into it while it is partly
+ *    filled; a full shared block is never copied (see pa_pool_append). */
 
 typedef struct pa_pool pa_pool;
 
@@ -213,8 +231,26 @@ void pa_pool_destroy(pa_pool* pool);
 int pa_pool_add_seq(pa_pool* pool, int64_t seq_id, const int32_t* token_ids, int32_t num_tokens,
                     int32_t* num_cached_tokens);
 
-/* Grow a sequence by n_new tokens; slots_out[n_new] receives their flat slots. */
+/* Grow a sequence by n_new tokens; slots_out[n_new] receives their flat slots.
+ * Copy-on-write: if n_new > 0 and the sequence's last block is partly filled
+ * and shared (ref_cnt > 1, after pa_pool_fork), the sequence first moves to
+ * a block popped from the head of the free queue; the pair (shared block,
+ * new block) is queued for pa_pool_take_copies, the shared block's ref_cnt
+ * drops by one, and the new tokens go to the new block.  That block counts
+ * toward the all-or-nothing check. */
 int pa_pool_append(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slots_out);
+
+/* Fork: child_id becomes a sequence with parent_id's length and block
+ * table; every block's ref_cnt rises by one (the blocks are shared, copy on
+ * write).  PA_ERR_INVALID_ARG if the parent is unknown or the child exists. */
+int pa_pool_fork(pa_pool* pool, int64_t parent_id, int64_t child_id);
+
+/* The block copies that copy-on-write queued, oldest first: src[i] is the
+ * shared block, dst[i] its new copy.  *n receives the count and the queue is
+ * emptied; PA_ERR_INVALID_ARG if cap < count (*n is still set, the queue
+ * kept).  Run them on the device with pa_copy_blocks before the
+ * pa_cache_write of the tokens that pa_pool_append placed in the copies. */
+int pa_pool_take_copies(pa_pool* pool, int32_t* src, int32_t* dst, int32_t cap, int32_t* n);
 
 /* Flat slots of positions [start, start + n) of a sequence (all < its length). */
 int pa_pool_slots(const pa_pool* pool, int64_t seq_id, int32_t start, int32_t n, int64_t* slots_out);

@@ -95,6 +95,15 @@ def pa_cache_write(desc, k_new, v_new, slot_mapping, k_cache, v_cache, stream=No
                                 _ptr(k_cache), _ptr(v_cache), _stream(stream)), "pa_cache_write")
 
 
+def pa_copy_blocks(desc, src, dst, k_cache, v_cache, stream=None):
+    """Copy-on-write's device half: K/V block dst[i] := block src[i] (int32 device tensors)."""
+    n = int(src.shape[0])
+    if int(dst.shape[0]) != n:
+        raise PaError(1, "pa_copy_blocks: src and dst differ in length")
+    _check(lib().pa_copy_blocks(ctypes.byref(desc), _ptr(src), _ptr(dst), n, _ptr(k_cache), _ptr(v_cache),
+                                _stream(stream)), "pa_copy_blocks")
+
+
 def pa_decode_workspace_size(desc, num_seqs) -> int:
     n = int(lib().pa_decode_workspace_size(ctypes.byref(desc), int(num_seqs)))
     if n == 0:
@@ -155,7 +164,8 @@ def default_scale(head_dim):
 
 
 class BlockPool:
-    """Host block pool (pa_pool_*): free_block_queue, ref_cnt, prefix sharing."""
+    """Host block pool (pa_pool_*): free_block_queue, ref_cnt, prefix sharing,
+    fork with copy-on-write."""
 
     def __init__(self, num_blocks, block_size, initial_free_order=None):
         self._lib = lib()
@@ -197,6 +207,19 @@ class BlockPool:
         out = (ctypes.c_int64 * max(1, n_new))()
         _check(self._lib.pa_pool_append(self._h, int(seq_id), int(n_new), out), "pa_pool_append")
         return list(out[:n_new])
+
+    def fork(self, parent_id, child_id):
+        """child_id shares every block of parent_id (copy on write)."""
+        _check(self._lib.pa_pool_fork(self._h, int(parent_id), int(child_id)), "pa_pool_fork")
+
+    def take_copies(self):
+        """The (src, dst) block copies queued by copy-on-write, oldest first."""
+        n = ctypes.c_int32()
+        self._lib.pa_pool_take_copies(self._h, None, None, 0, ctypes.byref(n))
+        src = (ctypes.c_int32 * max(1, n.value))()
+        dst = (ctypes.c_int32 * max(1, n.value))()
+        _check(self._lib.pa_pool_take_copies(self._h, src, dst, n.value, ctypes.byref(n)), "pa_pool_take_copies")
+        return [(src[i], dst[i]) for i in range(n.value)]
 
     def slots(self, seq_id, start, n):
         out = (ctypes.c_int64 * max(1, n))()

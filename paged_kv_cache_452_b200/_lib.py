@@ -15,6 +15,7 @@ SIGNATURES = {
     "pa_version": (ctypes.c_char_p, []),
     "pa_block_bytes": (_SZ, [_P]),
     "pa_cache_write": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _P, _P]),
+    "pa_copy_blocks": (ctypes.c_int, [_P, _P, _P, _I32, _P, _P, _P]),
     "pa_decode_workspace_size": (_SZ, [_P, _I32]),
     "pa_decode": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P, _SZ, _P]),
     "pa_decode_static": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P]),
@@ -25,6 +26,8 @@ SIGNATURES = {
     "pa_pool_destroy": (None, [_P]),
     "pa_pool_add_seq": (ctypes.c_int, [_P, _I64, _P, _I32, _P]),
     "pa_pool_append": (ctypes.c_int, [_P, _I64, _I32, _P]),
+    "pa_pool_fork": (ctypes.c_int, [_P, _I64, _I64]),
+    "pa_pool_take_copies": (ctypes.c_int, [_P, _P, _P, _I32, _P]),
     "pa_pool_slots": (ctypes.c_int, [_P, _I64, _I32, _I32, _P]),
     "pa_pool_free_seq": (ctypes.c_int, [_P, _I64]),
     "pa_pool_block_table": (ctypes.c_int, [_P, _I64, _P, _I32, _P]),

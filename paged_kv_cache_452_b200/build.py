@@ -20,7 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libpa.so")
-SOURCES = ["api.cu", "cache_write.cu", "decode_tc.cu", "attn_simt.cu", "prefill_tc.cu", "prefill_umma.cu", "decode_noalloc.cu", "pool.cpp"]
+SOURCES = ["api.cu", "cache_write.cu", "decode_tc.cu", "attn_simt.cu", "prefill_tc.cu", "prefill_umma.cu", "decode_noalloc.cu", "block_copy.cu", "pool.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

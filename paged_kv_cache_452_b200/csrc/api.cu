@@ -300,6 +300,29 @@ int pa_cache_write(const pa_cache_desc* d, const void* k_new, const void* v_new,
                      "pa_cache_write");
 }
 
+int pa_copy_blocks(const pa_cache_desc* d, const int32_t* src, const int32_t* dst, int32_t n, void* k_cache,
+                   void* v_cache, void* stream) {
+  clear_error();
+  int rc = check_desc(d, "pa_copy_blocks");
+  if (rc) return rc;
+  if (n < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: n < 0");
+  if (n == 0) return PA_OK;
+  if (!src || !dst || !k_cache || !v_cache) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: NULL pointer");
+  if (!aligned(src, 4) || !aligned(dst, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: misaligned pointer");
+  int sms = 0;
+  if ((rc = num_sms(&sms))) return rc;
+  CopyBlocksParams p = {};
+  p.src = src;
+  p.dst = dst;
+  p.n = n;
+  p.num_blocks = d->num_blocks;
+  p.block_bytes = (int64_t)(pa_block_bytes(d) / 2);
+  p.k_cache = static_cast<uint8_t*>(k_cache);
+  p.v_cache = static_cast<uint8_t*>(v_cache);
+  return cuda_status(launch_copy_blocks(p, sms, static_cast<cudaStream_t>(stream)), "pa_copy_blocks");
+}
+
 size_t pa_decode_workspace_size(const pa_cache_desc* d, int32_t num_seqs) {
   clear_error();
   if (check_desc(d, "pa_decode_workspace_size") || num_seqs < 0) return 0;

@@ -22,6 +22,20 @@ struct CacheWriteParams {
 };
 cudaError_t launch_cache_write(const CacheWriteParams& p, int in_dtype, int kv_dtype, cudaStream_t stream);
 
+// Whole-block copies inside both pools (copy-on-write): K and V block dst[i]
+// become copies of block src[i]; pairs with an id outside [0, num_blocks)
+// or src == dst are skipped.
+struct CopyBlocksParams {
+  const int32_t* src;
+  const int32_t* dst;
+  int32_t n;
+  int32_t num_blocks;
+  int64_t block_bytes;  // bytes of one block of one pool
+  uint8_t* k_cache;
+  uint8_t* v_cache;
+};
+cudaError_t launch_copy_blocks(const CopyBlocksParams& p, int num_sms, cudaStream_t stream);
+
 // Rows of a decode or mixed step.  Sequence s owns query rows
 // qsl[s] .. qsl[s+1]-1 (qsl == nullptr: exactly row s), the last of which
 // sits at position seq_lens[s] - 1.

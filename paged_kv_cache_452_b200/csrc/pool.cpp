@@ -3,8 +3,11 @@
 // The block manager described on "PagedAttention：KV cache 即虚拟内存（block
 // manager & 碎片）", section 深入原理 (V1 结构, 生命周期, 共享 → prefix caching),
 // with the allocation rule of the block-table snippet on "49 vLLM /
-// PagedAttention" (a new block when the token being appended starts one).
-// It only produces block tables and slots; it never touches KV bytes.
+// PagedAttention" (a new block when the token being appended starts one),
+// and copy-on-write for forked sequences (the same sharing bullet: a fork
+// that diverges inside a shared block triggers a copy; "49 vLLM /
+// PagedAttention", Почему это важно).  It only produces block tables, slots
+// and the list of block copies; it never touches KV bytes.
 //
 // free_block_queue is an intrusive doubly linked list over block ids (prev/
 // next arrays), so pop-head, push-tail and unlinking a parked block that a
@@ -61,6 +64,8 @@ struct pa_pool {
   std::vector<std::vector<int32_t>> toks;  // its token ids (for collision checks)
   std::unordered_map<uint64_t, int32_t> hash_to_block;
   std::unordered_map<int64_t, Seq> seqs;
+  // copy-on-write pairs (shared block, its new copy) for the caller to run
+  std::vector<int32_t> copy_src, copy_dst;
 
   void push_tail(int32_t b) {
     prev[b] = tail;
@@ -199,15 +204,56 @@ int pa_pool_append(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slots_
   const int64_t start = seq.num_tokens;
   const int64_t end = start + n_new;
   if (end > INT32_MAX) return pa::fail(PA_ERR_INVALID_ARG, "pa_pool_append: length overflow");
-  const int64_t need = (end + bs - 1) / bs - (int64_t)seq.blocks.size();
+  // writing into a partly filled last block that another sequence shares:
+  // move to a copy of it first
+  const bool cow = n_new > 0 && start % bs != 0 && pool->ref_cnt[seq.blocks.back()] > 1;
+  const int64_t need = (end + bs - 1) / bs - (int64_t)seq.blocks.size() + (cow ? 1 : 0);
   if (need > pool->nfree)
     return pa::fail(PA_ERR_NO_BLOCKS, "pa_pool_append: need %lld blocks, %d free", (long long)need,
                     pool->nfree);
+  if (cow) {
+    const int32_t src = seq.blocks.back();
+    const int32_t dst = pool->pop_head();
+    --pool->ref_cnt[src];
+    seq.blocks.back() = dst;
+    pool->copy_src.push_back(src);
+    pool->copy_dst.push_back(dst);
+  }
   for (int64_t p = start; p < end; ++p) {
     if ((int64_t)seq.blocks.size() * bs <= p) seq.blocks.push_back(pool->pop_head());
     slots_out[p - start] = (int64_t)seq.blocks[p / bs] * bs + p % bs;
   }
   seq.num_tokens = (int32_t)end;
+  return PA_OK;
+}
+
+int pa_pool_fork(pa_pool* pool, int64_t parent_id, int64_t child_id) {
+  pa::clear_error();
+  if (!pool) return pa::fail(PA_ERR_INVALID_ARG, "pa_pool_fork: pool is NULL");
+  auto it = pool->seqs.find(parent_id);
+  if (it == pool->seqs.end())
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_pool_fork: unknown sequence %lld", (long long)parent_id);
+  if (pool->seqs.count(child_id))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_pool_fork: sequence %lld exists", (long long)child_id);
+  Seq child = it->second;  // same length and blocks
+  for (int32_t b : child.blocks) ++pool->ref_cnt[b];
+  pool->seqs.emplace(child_id, std::move(child));
+  return PA_OK;
+}
+
+int pa_pool_take_copies(pa_pool* pool, int32_t* src, int32_t* dst, int32_t cap, int32_t* n) {
+  pa::clear_error();
+  if (!pool || !n) return pa::fail(PA_ERR_INVALID_ARG, "pa_pool_take_copies: NULL argument");
+  const size_t k = pool->copy_src.size();
+  *n = (int32_t)k;
+  if ((int64_t)k > cap || (k > 0 && (!src || !dst)))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_pool_take_copies: capacity %d < %zu", cap, k);
+  if (k > 0) {
+    std::memcpy(src, pool->copy_src.data(), sizeof(int32_t) * k);
+    std::memcpy(dst, pool->copy_dst.data(), sizeof(int32_t) * k);
+  }
+  pool->copy_src.clear();
+  pool->copy_dst.clear();
   return PA_OK;
 }
 

@@ -58,6 +58,33 @@ def test_scripted_trace_matches_model():
     same_state(c, m)
 
 
+def test_fork_and_copy_on_write_trace_matches_model():
+    order = [6, 2, 5, 0, 7, 1, 3, 4]
+    c, m = BlockPool(8, 4, order), BlockPoolModel(8, 4, order)
+    both(c, m, "add_seq", 1, 6, None)
+    both(c, m, "fork", 1, 2)
+    same_state(c, m)
+    both(c, m, "append", 2, 1)  # copy-on-write of the half-full shared block
+    assert both(c, m, "take_copies") is None
+    both(c, m, "append", 1, 2)
+    both(c, m, "fork", 1, 3)
+    both(c, m, "append", 3, 1)  # the shared block is full: no copy
+    both(c, m, "take_copies")
+    same_state(c, m)
+    assert both(c, m, "fork", 1, 3) == 1  # the child exists
+    assert both(c, m, "fork", 99, 5) == 1  # no such parent
+    both(c, m, "free_seq", 2)
+    both(c, m, "free_seq", 1)
+    same_state(c, m)
+    # no free block left for the copy: all-or-nothing
+    c2, m2 = BlockPool(2, 4), BlockPoolModel(2, 4)
+    both(c2, m2, "add_seq", 1, 5, None)
+    both(c2, m2, "fork", 1, 2)
+    assert both(c2, m2, "append", 2, 1) == 3
+    assert both(c2, m2, "take_copies") is None
+    same_state(c2, m2)
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_random_traces_match_model(seed):
     g = np.random.default_rng(seed)
@@ -67,7 +94,7 @@ def test_random_traces_match_model(seed):
     prefixes = [g.integers(0, 5, size=3 * bs).tolist() for _ in range(3)]
     live, next_id = [], 0
     for _ in range(400):
-        op = g.integers(0, 4)
+        op = g.integers(0, 6)
         if op == 0 or not live:
             n = int(g.integers(0, 4 * bs))
             toks = None
@@ -83,12 +110,18 @@ def test_random_traces_match_model(seed):
         elif op == 2:
             sid = live.pop(int(g.integers(0, len(live))))
             both(c, m, "free_seq", sid)
-        else:
+        elif op == 3:
             sid = live[int(g.integers(0, len(live)))]
             n = m.num_tokens(sid)
             if n:
                 a = int(g.integers(0, n))
                 both(c, m, "slots", sid, a, int(g.integers(0, n - a + 1)))
+        elif op == 4:  # fork; appends to either side then copy on write
+            if both(c, m, "fork", live[int(g.integers(0, len(live)))], next_id) is None:
+                live.append(next_id)
+            next_id += 1
+        else:
+            both(c, m, "take_copies")
         same_state(c, m)
 
 
