@@ -66,6 +66,37 @@ def test_cache_write_rejects_bad_arguments_on_host():
     assert _call_write(no_scale) == 1
 
 
+def test_copy_blocks_rejects_bad_arguments_on_host():
+    desc = pa.CacheDesc.make(16, 16, 2, 8, 128, "bf16", "bf16")
+    L = pa.lib()
+    p = 256
+    assert L.pa_copy_blocks(None, p, p, 1, p, p, None) == 1
+    assert L.pa_copy_blocks(ctypes.byref(desc), p, p, -1, p, p, None) == 1
+    assert L.pa_copy_blocks(ctypes.byref(desc), p, p, 0, p, p, None) == 0  # nothing to copy, nothing launched
+    assert L.pa_copy_blocks(ctypes.byref(desc), None, p, 2, p, p, None) == 1
+    assert b"NULL" in L.pa_last_error()
+    assert L.pa_copy_blocks(ctypes.byref(desc), p + 2, p, 2, p, p, None) == 1  # int32 ids misaligned
+    assert L.pa_copy_blocks(ctypes.byref(desc), p, p, 2, p, p + 8, None) == 1  # pool not 16-byte aligned
+    assert b"misaligned" in L.pa_last_error()
+
+
+def test_pool_fork_and_copy_queue_errors():
+    pool = pa.BlockPool(4, 4)
+    with pytest.raises(pa.PaError) as e:
+        pool.fork(1, 2)  # no parent
+    assert e.value.code == 1
+    pool.add_seq(1, 3)
+    pool.fork(1, 2)
+    with pytest.raises(pa.PaError):
+        pool.fork(1, 2)  # the child exists
+    pool.append(2, 1)  # copy-on-write of the shared, partly filled block
+    L = pa.lib()
+    n = ctypes.c_int32()
+    assert L.pa_pool_take_copies(pool._h, None, None, 0, ctypes.byref(n)) == 1 and n.value == 1
+    assert pool.take_copies() == [(0, 1)]  # kept after the refusal; block 1 is next in the queue
+    assert pool.take_copies() == []
+
+
 def test_decode_rejects_bad_arguments_on_host():
     desc = pa.CacheDesc.make(16, 16, 2, 8, 128, "bf16", "bf16")
     L = pa.lib()
