@@ -70,13 +70,15 @@ def test_single_process_needs_no_process_group():
         os.environ.update(env)
 
 
-def test_reference_arm_under_torchrun_two_ranks():
-    """`bench.py --impl reference` launched exactly as the driver launches an
-    N = 2 run: rank 0 alone times the oracle and prints one JSON line; rank 1
-    exits 0 without output."""
+@pytest.mark.parametrize("workload,metric", [("gqa_bf16", "paged decode attention KV GB/s"),
+                                             ("block_copy", "block copy GB/s")])
+def test_reference_arm_under_torchrun_two_ranks(workload, metric):
+    """`bench.py --impl reference` launched as an N = 2 run is launched:
+    rank 0 alone times the oracle and prints one JSON line; rank 1 exits 0
+    without output."""
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
-           "--gpus", "2", "--steps", "2", "--warmup", "3", "--ref-budget", "0.05", "--workload", "gqa_bf16"]
+           "--gpus", "2", "--steps", "2", "--warmup", "3", "--ref-budget", "0.05", "--workload", workload]
     env = dict(os.environ, OMP_NUM_THREADS="2")
     p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
     assert p.returncode == 0, p.stderr[-3000:]
@@ -86,3 +88,4 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 2 and d["warmup"] == 3
     assert d["value"] > 0 and d["unit"] == "GB/s" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["metric"] == metric and d["config"]["workload"] == workload
