@@ -367,8 +367,8 @@ def bench_ours(args):
     errs = [pa.workspace_error(b.workspace) for b in batches]
     if any(errs):
         raise SystemExit(f"kernel error word set: {errs}")
-    for gg in g_step + g_attend:
-        del gg
+    g_step.clear()  # release the graphs before the process group
+    g_attend.clear()
 
     if rank != 0:
         if world > 1:
@@ -529,8 +529,7 @@ def bench_block_copy(args):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = reduce_max(_time(e2e_step, args.steps, stream), world, device)
-    for gr in graphs:
-        del gr
+    graphs.clear()
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
