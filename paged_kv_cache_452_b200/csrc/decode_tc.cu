@@ -10,7 +10,7 @@
 // How, on sm_100a:
 //  * Work = (sequence, kv head, block) tiles.  The tiles of the whole batch
 //    are laid end to end and cut into one equal, contiguous range per warp
-//    (persistent grid, 2 CTAs of 4 warps per SM), so a long context is split
+//    (persistent grid, 3 CTAs of 4 warps per SM), so a long context is split
 //    over several warps (split-K over blocks) and every warp streams the
 //    same number of bytes whatever the length mix.  Each warp works alone:
 //    a (sequence, kv head) that lies wholly in its range is finished in
