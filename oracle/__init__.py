@@ -48,10 +48,10 @@ def lib():
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_cache_write.restype = c_i
         L.oracle_cache_write.argtypes = [c_i, c_i, c_p, c_p, c_p, c_i, c_i, c_i, c_i, c_i,
-                                         ctypes.c_float, ctypes.c_float, c_p, c_p]
+                                         ctypes.c_float, ctypes.c_float, c_p, c_p, c_p, c_p]
         L.oracle_attention.restype = None
         L.oracle_attention.argtypes = [c_p, c_i, c_p, c_p, c_p, c_i, c_i, c_p, c_p,
-                                       ctypes.c_double, ctypes.c_double, c_i, c_i, c_i, c_i,
+                                       ctypes.c_double, ctypes.c_double, c_p, c_p, c_i, c_i, c_i, c_i,
                                        ctypes.c_double, c_p, c_i]
         L.oracle_max_threads.restype = c_i
         _lib = L
@@ -78,6 +78,17 @@ def e4m3_encode(x) -> np.ndarray:
     x = np.asarray(x, dtype=np.float32)
     f = lib().oracle_e4m3_encode
     return np.array([f(float(v)) for v in x.ravel()], dtype=np.uint8).reshape(x.shape)
+
+
+def _scale_args(scale, num_kv_heads):
+    """(fp32 scalar, per-head fp32 array or None) for a scale given as one
+    number for the pool or as one number per kv head; the array is kept
+    alive by the caller while the C call runs."""
+    a = np.asarray(scale, dtype=np.float32)
+    if a.ndim == 0:
+        return float(a), None
+    assert a.shape == (num_kv_heads,), a.shape
+    return 1.0, np.ascontiguousarray(a)
 
 
 def new_cache(num_blocks, num_kv_heads, block_size, head_dim, kv_dtype, d_major=False):
@@ -108,7 +119,8 @@ def cache_write(k_new, v_new, slot_mapping, k_cache, v_cache, in_dtype, kv_dtype
     k_new, v_new: [T][Hkv][D] raw storage (float32 array for fp32, uint16 bits
     for bf16).  slot_mapping: int64 [T]; a negative slot is skipped.
     k_cache is [NB][Hkv][bs][D]; v_cache is too, except for e4m3 where it is
-    d-major [NB][Hkv][D][bs].
+    d-major [NB][Hkv][D][bs].  k_scale / v_scale: one fp32 number for the
+    pool, or one per kv head.
     """
     k_new = np.ascontiguousarray(k_new)
     v_new = np.ascontiguousarray(v_new)
@@ -118,9 +130,12 @@ def cache_write(k_new, v_new, slot_mapping, k_cache, v_cache, in_dtype, kv_dtype
     assert v_cache.shape == ((nb, hkv, d, bs) if kv_dtype == "e4m3" else (nb, hkv, bs, d))
     assert k_new.shape == (slots.shape[0], hkv, d), k_new.shape
     assert k_new.dtype == _NPDT[in_dtype] and k_cache.dtype == _NPDT[kv_dtype]
+    ks, kh = _scale_args(k_scale, hkv)
+    vs, vh = _scale_args(v_scale, hkv)
     rc = lib().oracle_cache_write(_DT[in_dtype], _DT[kv_dtype], _ptr(k_new), _ptr(v_new),
-                                  _ptr(slots), slots.shape[0], nb, bs, hkv, d,
-                                  float(k_scale), float(v_scale), _ptr(k_cache), _ptr(v_cache))
+                                  _ptr(slots), slots.shape[0], nb, bs, hkv, d, ks, vs,
+                                  None if kh is None else _ptr(kh), None if vh is None else _ptr(vh),
+                                  _ptr(k_cache), _ptr(v_cache))
     if rc != 0:
         raise ValueError("slot past the end of the pool")
 
@@ -144,8 +159,9 @@ def attention(q, row_seq, row_pos, block_tables, k_cache, v_cache, kv_dtype, num
     q: [R][Hq][D] (any float dtype; upcast to fp64 exactly).
     row_seq[r], row_pos[r]: sequence and position of row r; it attends keys
     0..row_pos[r].  block_tables: int32 [S][max_blocks].
-    k_scale / v_scale are the cache's fp32 per-tensor scales (an e4m3 code
-    dequantises to its value times the fp32 scale, in fp64).
+    k_scale / v_scale are the cache's fp32 scales, one number for the pool or
+    one per kv head (an e4m3 code dequantises to its value times its head's
+    fp32 scale, in fp64).
     Returns out [R][Hq][D] fp64.
     """
     q = np.ascontiguousarray(q, dtype=np.float64)
@@ -157,8 +173,10 @@ def attention(q, row_seq, row_pos, block_tables, k_cache, v_cache, kv_dtype, num
     r = q.shape[0]
     assert q.shape == (r, num_q_heads, d)
     out = np.empty((r, num_q_heads, d), dtype=np.float64)
+    ks, kh = _scale_args(k_scale, hkv)
+    vs, vh = _scale_args(v_scale, hkv)
     lib().oracle_attention(_ptr(q), r, _ptr(row_seq), _ptr(row_pos), _ptr(bt), bt.shape[1],
-                           _DT[kv_dtype], _ptr(k_cache), _ptr(v_cache),
-                           float(np.float32(k_scale)), float(np.float32(v_scale)), bs, num_q_heads, hkv, d, float(scale), _ptr(out),
-                           int(num_threads))
+                           _DT[kv_dtype], _ptr(k_cache), _ptr(v_cache), ks, vs,
+                           None if kh is None else _ptr(kh), None if vh is None else _ptr(vh),
+                           bs, num_q_heads, hkv, d, float(scale), _ptr(out), int(num_threads))
     return out

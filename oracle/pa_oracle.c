@@ -14,7 +14,10 @@
  *    пейджинга)"), with the new token's flat slot split into (physical block,
  *    offset) = (slot / block_size, slot % block_size).  fp32/bf16 caches get a
  *    byte copy; an FP8 cache gets e4m3(fp32(x) / fp32(scale)), rounded to
- *    nearest-even and saturated to +-448.
+ *    nearest-even and saturated to +-448.  The scale is one fp32 per pool,
+ *    or one per kv head (this build's reading: the pages motivate FP8 KV,
+ *    "PagedAttention：KV cache 即虚拟内存…", num_gpu_blocks and the KV-bound
+ *    question, halving the bytes per block, and leave the scale open).
  *
  *  - oracle_attention: attention over the keys a block table points at.  The
  *    page "PagedAttention：KV cache 即虚拟内存（block manager & 碎片）" states
@@ -130,10 +133,13 @@ static size_t orc_index(int d_major, size_t b, size_t h, size_t o, size_t d, int
 
 /* k_new, v_new: [num_tokens][num_kv_heads][head_dim] in in_dtype (fp32 or bf16).
  * k_cache, v_cache: the pools, laid out as described at the top of this file.
+ * k_head_scales, v_head_scales: NULL (k_scale / v_scale for every head) or
+ * one fp32 scale per kv head.
  * A negative slot is skipped.  Returns 0, or -1 if a slot is past the pool. */
 int oracle_cache_write(int in_dtype, int kv_dtype, const void* k_new, const void* v_new,
                        const int64_t* slots, int num_tokens, int num_blocks, int block_size,
                        int num_kv_heads, int head_dim, float k_scale, float v_scale,
+                       const float* k_head_scales, const float* v_head_scales,
                        void* k_cache, void* v_cache) {
   int t, h, d, side;
   for (t = 0; t < num_tokens; ++t) {
@@ -146,8 +152,9 @@ int oracle_cache_write(int in_dtype, int kv_dtype, const void* k_new, const void
     for (side = 0; side < 2; ++side) {
       const void* src = side == 0 ? k_new : v_new;
       void* dst = side == 0 ? k_cache : v_cache;
-      float scale = side == 0 ? k_scale : v_scale;
+      const float* head_scales = side == 0 ? k_head_scales : v_head_scales;
       for (h = 0; h < num_kv_heads; ++h) {
+        float scale = head_scales ? head_scales[h] : (side == 0 ? k_scale : v_scale);
         for (d = 0; d < head_dim; ++d) {
           size_t si = ((size_t)t * num_kv_heads + h) * head_dim + d;
           int d_major = (side == 1 && kv_dtype == ORC_E4M3);
@@ -176,12 +183,14 @@ int oracle_cache_write(int in_dtype, int kv_dtype, const void* k_new, const void
  * decode row sits at the last position, so it attends the whole context).
  * Query head h reads KV head h / (num_q_heads / num_kv_heads).
  * block_tables: [num_seqs][max_blocks] int32.
+ * An e4m3 code of kv head h dequantises to its value times k_head_scales[h]
+ * (v_head_scales[h] for V), or times k_scale (v_scale) when those are NULL.
  * out: [num_rows][num_q_heads][head_dim] fp64. */
 void oracle_attention(const double* q, int num_rows, const int32_t* row_seq, const int32_t* row_pos,
                       const int32_t* block_tables, int max_blocks, int kv_dtype, const void* k_cache,
-                      const void* v_cache, double k_scale, double v_scale, int block_size,
-                      int num_q_heads, int num_kv_heads, int head_dim, double scale, double* out,
-                      int num_threads) {
+                      const void* v_cache, double k_scale, double v_scale, const float* k_head_scales,
+                      const float* v_head_scales, int block_size, int num_q_heads, int num_kv_heads,
+                      int head_dim, double scale, double* out, int num_threads) {
   int group = num_q_heads / num_kv_heads;
   long task, ntasks = (long)num_rows * num_q_heads;
 #ifdef _OPENMP
@@ -192,6 +201,8 @@ void oracle_attention(const double* q, int num_rows, const int32_t* row_seq, con
     int r = (int)(task / num_q_heads);
     int h = (int)(task % num_q_heads);
     int kvh = h / group;
+    double ks = k_head_scales ? (double)k_head_scales[kvh] : k_scale;
+    double vs = v_head_scales ? (double)v_head_scales[kvh] : v_scale;
     int s = row_seq[r];
     int n = row_pos[r] + 1;
     const double* qv = q + ((size_t)r * num_q_heads + h) * head_dim;
@@ -206,7 +217,7 @@ void oracle_attention(const double* q, int num_rows, const int32_t* row_seq, con
       for (d = 0; d < head_dim; ++d)
         dot += qv[d] * orc_load_cache(k_cache, kv_dtype,
                                       orc_index(0, blk, kvh, off, d, num_kv_heads, block_size, head_dim),
-                                      k_scale);
+                                      ks);
       logit[j] = scale * dot;
       if (logit[j] > mx) mx = logit[j];
     }
@@ -220,7 +231,7 @@ void oracle_attention(const double* q, int num_rows, const int32_t* row_seq, con
         o[d] += w * orc_load_cache(v_cache, kv_dtype,
                                    orc_index(kv_dtype == ORC_E4M3, blk, kvh, off, d, num_kv_heads,
                                              block_size, head_dim),
-                                   v_scale);
+                                   vs);
     }
     free(logit);
   }

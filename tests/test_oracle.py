@@ -325,3 +325,71 @@ def test_fp8_attention_uses_dequantised_values():
         vd = np.stack([_torch_e4m3_value(vc[x // bs, :, :, x % bs]) for x in slots]) * np.float64(np.float32(vs))
         ref = _sdpa(q[s], kd, vd, 0.25, hq, hkv, n - 1)
         np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------- per-head fp8 scales
+
+def test_per_head_quantisation_matches_torch():
+    """One scale per kv head (amax of that head / 448): every code equals
+    torch's e4m3 cast of x / scale_h in fp32."""
+    nb, hkv, bs, d = 8, 4, 16, 32
+    g = np.random.default_rng(21)
+    mag = np.array([0.1, 1.0, 7.0, 300.0], dtype=np.float32)[None, :, None]  # very different heads
+    k = torch.from_numpy(g.standard_normal((40, hkv, d), dtype=np.float32) * mag).bfloat16()
+    v = torch.from_numpy(g.standard_normal((40, hkv, d), dtype=np.float32) * mag[:, ::-1]).bfloat16()
+    ks = (k.float().abs().amax(dim=(0, 2)) / 448).numpy().astype(np.float32)
+    vs = (v.float().abs().amax(dim=(0, 2)) / 448).numpy().astype(np.float32)
+    assert len(set(ks.tolist())) == hkv
+    kc, vc = oracle.new_caches(nb, hkv, bs, d, "e4m3")
+    slots = g.permutation(nb * bs)[:40]
+    oracle.cache_write(k.view(torch.int16).numpy().view(np.uint16), v.view(torch.int16).numpy().view(np.uint16),
+                       slots, kc, vc, "bf16", "e4m3", ks, vs)
+    kq = (k.float() / torch.from_numpy(ks)[None, :, None]).to(E4M3).view(torch.uint8).numpy()
+    vq = (v.float() / torch.from_numpy(vs)[None, :, None]).to(E4M3).view(torch.uint8).numpy()
+    for t, s in enumerate(slots):
+        assert np.array_equal(kc[s // bs, :, s % bs], kq[t])
+        assert np.array_equal(vc[s // bs, :, :, s % bs], vq[t])
+
+
+def test_per_head_scales_all_equal_give_the_per_tensor_bits():
+    lens = [23, 40]
+    hq, hkv, d, bs = 8, 2, 16, 16
+    P = _paged_problem(lens, hq, hkv, d, bs, seed=22)
+    q = np.random.default_rng(23).standard_normal((2, hq, d))
+    outs, caches = [], []
+    for ks, vs in ((0.03, 0.05), (np.full(hkv, 0.03, np.float32), np.full(hkv, 0.05, np.float32))):
+        kc, vc = oracle.new_caches(*P["kc"].shape, "e4m3")
+        for s, n in enumerate(lens):
+            slots = np.array([P["tables"][s, p // bs] * bs + p % bs for p in range(n)])
+            oracle.cache_write(P["ks"][s], P["vs"][s], slots, kc, vc, "f32", "e4m3", ks, vs)
+        caches.append((kc, vc))
+        outs.append(oracle.attention(q, [0, 1], np.array(lens) - 1, P["tables"], kc, vc, "e4m3", hq, 0.25,
+                                     ks, vs))
+    assert np.array_equal(caches[0][0], caches[1][0]) and np.array_equal(caches[0][1], caches[1][1])
+    assert np.array_equal(outs[0], outs[1])
+
+
+def test_per_head_fp8_attention_uses_each_heads_scale():
+    """GQA group 2 over 2 kv heads with different scales: SDPA on the values
+    torch decodes from the same codes, each head times its own scale."""
+    lens = [20, 37]
+    hq, hkv, d, bs = 4, 2, 16, 16
+    P = _paged_problem(lens, hq, hkv, d, bs, seed=24)
+    ks = np.array([0.01, 0.004], dtype=np.float32)
+    vs = np.array([0.02, 0.05], dtype=np.float32)
+    kc, vc = oracle.new_caches(*P["kc"].shape, "e4m3")
+    for s, n in enumerate(lens):
+        slots = np.array([P["tables"][s, p // bs] * bs + p % bs for p in range(n)])
+        oracle.cache_write(P["ks"][s], P["vs"][s], slots, kc, vc, "f32", "e4m3", ks, vs)
+    q = np.random.default_rng(25).standard_normal((2, hq, d))
+    out = oracle.attention(q, [0, 1], np.array(lens) - 1, P["tables"], kc, vc, "e4m3", hq, 0.25, ks, vs)
+    for s, n in enumerate(lens):
+        slots = [P["tables"][s, p // bs] * bs + p % bs for p in range(n)]
+        kd = np.stack([_torch_e4m3_value(kc[x // bs, :, x % bs]) for x in slots]) * ks.astype(np.float64)[None, :, None]
+        vd = np.stack([_torch_e4m3_value(vc[x // bs, :, :, x % bs]) for x in slots]) * vs.astype(np.float64)[None, :, None]
+        ref = _sdpa(q[s], kd, vd, 0.25, hq, hkv, n - 1)
+        np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
+    # and the scales matter: swapping them changes the output
+    swapped = oracle.attention(q, [0, 1], np.array(lens) - 1, P["tables"], kc, vc, "e4m3", hq, 0.25,
+                               ks[::-1].copy(), vs[::-1].copy())
+    assert np.abs(swapped - out).max() > 1e-3
