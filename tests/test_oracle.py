@@ -240,6 +240,35 @@ def test_attention_matches_torch_sdpa_decode(hq, hkv, d, bs):
         np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
 
 
+def test_attention_over_a_bf16_cache_matches_torch_sdpa():
+    """The bf16 load path: K/V rounded to bf16 by torch, written as bf16 bits,
+    attended by the oracle = torch fp64 SDPA on torch's bf16 values."""
+    lens = [3, 16, 41]
+    hq, hkv, d, bs = 8, 2, 16, 16
+    g = np.random.default_rng(31)
+    nb = sum(-(-n // bs) for n in lens) + 2
+    tables = np.full((len(lens), max(-(-n // bs) for n in lens)), -1, dtype=np.int32)
+    phys = g.permutation(nb)
+    kc, vc = oracle.new_caches(nb, hkv, bs, d, "bf16")
+    kvals, vvals, pos = [], [], 0
+    for s, n in enumerate(lens):
+        m = -(-n // bs)
+        tables[s, :m] = phys[pos:pos + m]
+        pos += m
+        k = torch.from_numpy(g.standard_normal((n, hkv, d), dtype=np.float32)).bfloat16()
+        v = torch.from_numpy(g.standard_normal((n, hkv, d), dtype=np.float32)).bfloat16()
+        slots = np.array([tables[s, p // bs] * bs + p % bs for p in range(n)])
+        oracle.cache_write(k.view(torch.int16).numpy().view(np.uint16), v.view(torch.int16).numpy().view(np.uint16),
+                           slots, kc, vc, "bf16", "bf16")
+        kvals.append(k.double().numpy())
+        vvals.append(v.double().numpy())
+    q = g.standard_normal((len(lens), hq, d))
+    out = oracle.attention(q, np.arange(len(lens)), np.array(lens) - 1, tables, kc, vc, "bf16", hq, 0.25)
+    for s, n in enumerate(lens):
+        ref = _sdpa(q[s], kvals[s], vvals[s], 0.25, hq, hkv, n - 1)
+        np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
+
+
 def test_attention_matches_torch_sdpa_causal_rows():
     lens = [23, 50]
     hq, hkv, d, bs = 6, 3, 16, 8
