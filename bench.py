@@ -32,15 +32,16 @@ METRIC = "paged decode attention KV GB/s"
 DEFAULT_WORKLOAD = "gqa_bf16"
 
 # DRAM bytes (read + write) per launch of the workload's dominant kernel from
-# one ncu capture (profiles/), valid only for the kernel source that was
-# profiled: any edit to the source drops the figure to null.
+# one ncu capture of that kernel, valid only for the kernel source that was
+# profiled (keyed by its sha256): any edit to the source drops the figure to
+# null until the kernel is captured again.
 PROFILED_TRAFFIC = {
     "gqa_bf16": {"source": "paged_kv_cache_452_b200/csrc/decode_tc.cu",
                  # the captured source with its header comment's CTA count corrected
                  # (a comment-only edit, same line count; the code is unchanged)
                  "sha256": "faab74a6d10b8ea93dd8d701d95eb0efa43c2f4d3fba534abb49367ada175fa1",
                  "bytes": 294_643_200},
-    # profiles/copy_blocks_block_copy.md: mean of two launches
+    # mean of two captured launches
     "block_copy": {"source": "paged_kv_cache_452_b200/csrc/block_copy.cu",
                    "sha256": "14c4d4e16d7a6cfba5f9139645ec9d67aba270f8986a597db740b32a1a2c0f11",
                    "bytes": 488_925_056},
@@ -59,6 +60,8 @@ def profiled_traffic(workload):
     except OSError:
         return None
     return e["bytes"] if digest == e["sha256"] else None
+
+
 KV_BYTES = {"f32": 4, "bf16": 2, "e4m3": 1}
 Q_BYTES = {"f32": 4, "bf16": 2}
 
@@ -190,18 +193,22 @@ def oracle_time(prep):
 
 
 def oracle_sample(wl, budget_s):
-    """A prefix of the batch whose oracle evaluation takes about budget_s
-    (scaled from a timing of the first sequence); its KV bytes."""
+    """Sequences of the batch whose oracle evaluation takes about budget_s,
+    shortest first (the cost per token is scaled from a timing of the
+    shortest sequence); their KV bytes."""
     import oracle
-    t = oracle_time(oracle_prepare(wl, [0]))
-    per_token = t / max(1, int(wl.context_lens[0] + wl.q_lens[0]))
+    tokens = (wl.context_lens + wl.q_lens).astype(np.int64)
+    order = [int(s) for s in np.argsort(tokens, kind="stable")]
+    t = oracle_time(oracle_prepare(wl, [order[0]]))
+    per_token = t / max(1, int(tokens[order[0]]))
     seqs, est = [], 0.0
-    for s in range(wl.num_seqs):
-        n = int(wl.context_lens[s] + wl.q_lens[s])
+    for s in order:
+        n = int(tokens[s])
         if seqs and est + per_token * n > budget_s:
             break
         seqs.append(s)
         est += per_token * n
+    seqs.sort()
     kv = sum(int(wl.context_lens[s] + wl.q_lens[s]) for s in seqs) * 2 * wl.num_kv_heads * wl.head_dim * \
         KV_BYTES[wl.kv_dtype]
     return oracle_prepare(wl, seqs), len(seqs), kv, oracle.max_threads()
@@ -211,8 +218,8 @@ def cpu_baseline(wl, budget_s=15.0):
     prep, n, kv, cores = oracle_sample(wl, budget_s)
     t = oracle_time(prep)
     return {"value": kv / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} of {wl.num_seqs} sequences of {wl.name}: their cache writes and all their "
-                      f"query rows, fp64 C oracle, {t:.2f} s"}
+            "sample": f"the {n} shortest of {wl.num_seqs} sequences of {wl.name}: their cache writes and "
+                      f"all their query rows, fp64 C oracle, {t:.2f} s"}
 
 
 def bench_reference(args):
@@ -253,107 +260,250 @@ def _time(fn, steps, stream):
     return e0.elapsed_time(e1) / steps
 
 
-def bench_ours(args):
-    world, rank, local = dist_setup(args)
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    import paged_kv_cache_452_b200 as pa
-    from paged_kv_cache_452_b200 import runner
+# Untimed back-to-back replays just before the timed steps, so that the
+# nvidia-smi samples (taken every 50 ms) see the GPU under this load: a timed
+# region of 20 steps of 60 us is far shorter than one sampling interval.
+CLOCK_WINDOW_S = 0.3
 
-    wl = W.make(args.workload, "full")
-    # two copies of the pool, used alternately, so no step finds the previous
-    # step's K/V in L2 (each copy is larger than L2 already)
-    batches = [runner.setup(wl, device) for _ in range(2)]
-    alg_bytes, kv_bytes = algorithmic_bytes(wl)
-    stream = torch.cuda.current_stream()
 
-    # eager warm-up through the public API, then one CUDA graph per pool copy
-    # for the step (cache write + decode) and for the decode alone, as a
-    # serving loop would replay them
-    for i in range(args.warmup):
-        runner.step(batches[i & 1])
-    torch.cuda.synchronize()
-    g_step, g_attend = [], []
-    for b in batches:
-        gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gs):
-            runner.step(b)
-        with torch.cuda.graph(ga):
-            runner.attend(b)
-        g_step.append(gs)
-        g_attend.append(ga)
-    for i in range(args.warmup):
-        g_step[i & 1].replay()
-        g_attend[i & 1].replay()
-    torch.cuda.synchronize()
+def _load(seconds, fn):
+    t_end = time.perf_counter() + seconds
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(32):
+            fn(i)
+            i += 1
+        torch.cuda.synchronize()
 
-    sampler = ClockSampler(local) if rank == 0 else None
-    time.sleep(0.2 if sampler else 0)
-    barrier(world)
-    torch.cuda.synchronize()
-    ms = _time(lambda i: g_step[i & 1].replay(), args.steps, stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ms = reduce_max(ms, world, device)
-    # the dominant kernel, pa_decode's single launch, per launch: replays of a
-    # graph holding only it, events on the replay stream
-    attend_ms = reduce_max(_time(lambda i: g_attend[i & 1].replay(), args.steps, stream), world, device)
-    clocks = sampler.stop() if sampler else None
-    # the same step issued launch by launch from Python (no graph)
-    eager_ms = reduce_max(_time(lambda i: runner.step(batches[i & 1]), args.steps, stream), world, device)
 
-    # end to end through the public API with host buffers: every step copies
-    # its inputs from pinned host memory, runs write + attention, and reads
-    # its output back.  As a serving loop would, the copies of one step
-    # overlap the kernels of its neighbours: uploads on one stream, the
-    # kernels on the main stream, downloads on a third, two device input
-    # sets used alternately (the pool and the workspace are shared; the
-    # kernels stay in order on the main stream).
+def prefill_flops(wl):
+    """QK^T and PV FLOPs of the step's prompt rows (q_len > 1): 4 * Hq * D
+    per (query row, attended key), causal over prior context + chunk."""
+    f = 0
+    for c, q in zip(wl.context_lens.tolist(), wl.q_lens.tolist()):
+        if q > 1:
+            keys = q * c + q * (q + 1) // 2  # row i attends c + i + 1 keys
+            f += 4 * wl.num_q_heads * wl.head_dim * keys
+    return f
+
+
+def _fusable(desc):
+    """pa_decode_fused covers the tensor-core decode: bf16 queries, a bf16 or
+    e4m3 pool, GQA group 2..8."""
+    g = desc.num_q_heads // desc.num_kv_heads
+    return desc.q_dtype == 1 and 2 <= g <= 8 and desc.kv_dtype in (1, 2)
+
+
+class Measured:
+    """One workload's graph-replayed step and attention, timed on one rank
+    (max over ranks), with the clocks seen meanwhile."""
+
+    def __init__(self, wl, device, args, world, rank, local):
+        from paged_kv_cache_452_b200 import runner
+        self.wl = wl
+        b0 = runner.setup(wl, device)
+        # the second copy of the pool, used alternately with the first so no
+        # step finds the previous step's K/V in L2 (each copy is larger than L2)
+        self.batches = [b0, runner.clone(b0)]
+        stream = torch.cuda.current_stream()
+        # eager warm-up through the public API, then one CUDA graph per pool
+        # copy for the step (cache write + attention) and for the attention
+        # alone, as a serving loop would replay them
+        for i in range(args.warmup):
+            runner.step(self.batches[i & 1])
+        torch.cuda.synchronize()
+        self.g_step, self.g_attend = [], []
+        for b in self.batches:
+            gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs):
+                runner.step(b)
+            with torch.cuda.graph(ga):
+                runner.attend(b)
+            self.g_step.append(gs)
+            self.g_attend.append(ga)
+        # the same step as one launch (pa_decode_fused), where the path fuses it
+        self.g_fused = []
+        if int(wl.q_lens.max()) == 1 and _fusable(b0.desc):
+            for b in self.batches:
+                gf = torch.cuda.CUDAGraph()
+                runner.step_fused(b)
+                torch.cuda.synchronize()
+                with torch.cuda.graph(gf):
+                    runner.step_fused(b)
+                self.g_fused.append(gf)
+        # shared prefixes attended once for their sequences (pa_decode_prefix)
+        self.g_pstep, self.g_pattend, self.plans = [], [], []
+        if wl.sharing is not None or getattr(wl, "prefix_group", None) is not None:
+            for b in self.batches:
+                plan = runner.prefix_plan(b)
+                if plan.groups.num_prefixes == 0:
+                    break
+                runner.step_prefix(b, plan)
+                torch.cuda.synchronize()
+                gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gs):
+                    runner.step_prefix(b, plan)
+                with torch.cuda.graph(ga):
+                    runner.attend_prefix(b, plan)
+                self.plans.append(plan)
+                self.g_pstep.append(gs)
+                self.g_pattend.append(ga)
+        for i in range(args.warmup):
+            self.g_step[i & 1].replay()
+            self.g_attend[i & 1].replay()
+            if self.g_fused:
+                self.g_fused[i & 1].replay()
+            if self.g_pstep:
+                self.g_pstep[i & 1].replay()
+                self.g_pattend[i & 1].replay()
+        torch.cuda.synchronize()
+
+        sampler = ClockSampler(local) if rank == 0 else None
+        _load(CLOCK_WINDOW_S, lambda i: self.g_step[i & 1].replay())
+        barrier(world)
+        torch.cuda.synchronize()
+        ms = _time(lambda i: self.g_step[i & 1].replay(), args.steps, stream)
+        # the attention kernels alone: replays of a graph holding only them,
+        # events on the replay stream
+        attend_ms = _time(lambda i: self.g_attend[i & 1].replay(), args.steps, stream)
+        fused_ms = _time(lambda i: self.g_fused[i & 1].replay(), args.steps, stream) if self.g_fused else None
+        pstep_ms = _time(lambda i: self.g_pstep[i & 1].replay(), args.steps, stream) if self.g_pstep else None
+        pattend_ms = _time(lambda i: self.g_pattend[i & 1].replay(), args.steps, stream) if self.g_pstep else None
+        torch.cuda.synchronize()
+        barrier(world)
+        self.clocks = sampler.stop() if sampler else None
+        self.ms = reduce_max(ms, world, device)
+        self.attend_ms = reduce_max(attend_ms, world, device)
+        self.fused_ms = reduce_max(fused_ms, world, device) if fused_ms is not None else None
+        self.pstep_ms = reduce_max(pstep_ms, world, device) if pstep_ms is not None else None
+        self.pattend_ms = reduce_max(pattend_ms, world, device) if pattend_ms is not None else None
+        self.alg_bytes, self.kv_bytes = algorithmic_bytes(wl)
+
+    def check(self):
+        import paged_kv_cache_452_b200 as pa
+        errs = [pa.workspace_error(b.workspace) for b in self.batches]
+        errs += [pa.workspace_error(pl.workspace) for pl in self.plans]
+        if any(errs):
+            raise SystemExit(f"{self.wl.name}: kernel error word set: {errs}")
+
+    def release(self):
+        self.g_step.clear()
+        self.g_attend.clear()
+        self.g_fused.clear()
+        self.g_pstep.clear()
+        self.g_pattend.clear()
+        self.plans.clear()
+        self.batches.clear()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    def summary(self, world, hbm, tc_peak):
+        wl = self.wl
+        rows = wl.num_new_tokens
+        decode_rows = int((wl.q_lens == 1).sum())
+        kv_gbs = self.alg_bytes / (self.attend_ms * 1e-3) / 1e9
+        d = {"workload": wl.name, "num_seqs": wl.num_seqs, "query_rows": rows, "decode_rows": decode_rows,
+             "kv_dtype": wl.kv_dtype, "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
+             "head_dim": wl.head_dim, "block_size": wl.block_size,
+             "context_tokens": int((wl.context_lens + wl.q_lens).sum()),
+             "algorithmic_bytes": self.alg_bytes, "kv_bytes": self.kv_bytes,
+             "attend_us": self.attend_ms * 1e3, "step_us": self.ms * 1e3,
+             "kv_gbs": world * kv_gbs, "frac_of_measured_hbm": kv_gbs / hbm, "frac_of_8tbs": kv_gbs / 8000.0,
+             "step_gbs": job_throughput(world, self.alg_bytes, self.ms),
+             "tokens_per_s": world * rows / (self.ms * 1e-3),
+             "decode_tokens_per_s": world * decode_rows / (self.ms * 1e-3),
+             "clocks": self.clocks}
+        if self.fused_ms is not None:  # write + attention in one launch
+            d["fused_step_us"] = self.fused_ms * 1e3
+            d["fused_step_gbs"] = job_throughput(world, self.alg_bytes, self.fused_ms)
+        if self.pstep_ms is not None:  # shared prefixes attended once (pa_decode_prefix)
+            d["prefix_path_attend_us"] = self.pattend_ms * 1e3
+            d["prefix_path_step_us"] = self.pstep_ms * 1e3
+            d["prefix_path_kv_gbs"] = world * self.alg_bytes / (self.pattend_ms * 1e-3) / 1e9
+        if wl.sharing is not None:  # the shared prefix counted once per sequence
+            d["logical_kv_bytes"] = logical_kv_bytes(wl)
+            d["effective_gbs"] = world * logical_kv_bytes(wl) / (self.attend_ms * 1e-3) / 1e9
+        flops = prefill_flops(wl)
+        if flops:
+            # the step's bound: its bytes at the copy peak or its prompt-row
+            # FLOPs at the sustained bf16 tensor peak, whichever is slower
+            bound_us = max(self.alg_bytes / (hbm * 1e9), flops / (tc_peak * 1e12)) * 1e6
+            d.update({"prefill_flops": flops, "bound_us": bound_us, "frac_of_bound": bound_us / (self.ms * 1e3)})
+        return d
+
+
+def e2e_measure(m, device, args, world):
+    """End to end through the public API with host buffers: every step
+    uploads its inputs from pinned host memory (one packed copy), runs cache
+    write + attention (a CUDA graph captured from the public calls, replayed
+    once per step) and reads its output back.  Uploads run on one stream and
+    downloads on another, two device input sets used alternately, so a
+    step's copies overlap its neighbours' kernels; the kernels stay in order
+    on the main stream (two attention grids never run at once)."""
     import copy
-    b0 = batches[0]
+
+    from paged_kv_cache_452_b200 import runner
     keys = ("q", "k_new", "v_new", "slots", "tables", "seq_lens")
-    host = {k: getattr(b0, k).cpu().pin_memory() for k in keys}
-    out_host = [torch.empty(b0.out.shape, dtype=b0.out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host[0].numel() * out_host[0].element_size()
-    sets = []
-    for _ in range(2):
-        st = copy.copy(b0)
-        for k in keys:
-            setattr(st, k, torch.empty_like(getattr(b0, k)))
+    b0 = m.batches[0]
+    layout, off = {}, 0
+    for k in keys:
+        t = getattr(b0, k)
+        n = t.numel() * t.element_size()
+        layout[k] = (off, n, t.dtype, tuple(t.shape))
+        off += (n + 255) // 256 * 256
+    host = torch.empty(off, dtype=torch.uint8).pin_memory()
+    for k, (o, n, _, _) in layout.items():
+        host[o:o + n].copy_(getattr(b0, k).detach().cpu().contiguous().view(-1).view(torch.uint8))
+    stream = torch.cuda.current_stream()
+    sets, devbufs, graphs = [], [], []
+    for j in range(2):
+        buf = torch.empty(off, dtype=torch.uint8, device=device)
+        st = copy.copy(m.batches[j])  # pool copy j and its workspace
+        for k, (o, n, dt, shape) in layout.items():
+            setattr(st, k, buf[o:o + n].view(dt).view(shape))
         st.out = torch.empty_like(b0.out)
+        buf.copy_(host)
+        torch.cuda.synchronize()
+        runner.step(st)  # the set's tensor maps and launch attributes are set up before capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            runner.step(st)
         sets.append(st)
+        devbufs.append(buf)
+        graphs.append(g)
+    out_host = [torch.empty(b0.out.shape, dtype=b0.out.dtype).pin_memory() for _ in range(2)]
+    d2h = out_host[0].numel() * out_host[0].element_size()
     up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
     landed = [torch.cuda.Event() for _ in range(2)]    # a set's inputs are on the device
     computed = [torch.cuda.Event() for _ in range(2)]  # a set's kernels have run
     read = [torch.cuda.Event() for _ in range(2)]      # a set's output is on the host
+    for j in range(2):
+        computed[j].record(stream)
+        read[j].record(stream)
 
-    def e2e_step(i):
+    def step(i):
         j = i & 1
-        st = sets[j]
         with torch.cuda.stream(up):
             up.wait_event(computed[j])  # the set's previous kernels no longer need its inputs
-            for k, t in host.items():
-                getattr(st, k).copy_(t, non_blocking=True)
+            devbufs[j].copy_(host, non_blocking=True)
             landed[j].record(up)
         stream.wait_event(landed[j])
         stream.wait_event(read[j])  # the set's previous output has been read
-        runner.step(st)
+        graphs[j].replay()
         computed[j].record(stream)
         with torch.cuda.stream(down):
             down.wait_event(computed[j])
-            out_host[j].copy_(st.out, non_blocking=True)
+            out_host[j].copy_(sets[j].out, non_blocking=True)
             read[j].record(down)
 
-    def e2e_time(steps):
+    def timed(steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         up.wait_event(e0)
         down.wait_event(e0)
         for i in range(steps):
-            e2e_step(i)
+            step(i)
         stream.wait_stream(up)
         stream.wait_stream(down)
         e1.record(stream)
@@ -361,50 +511,96 @@ def bench_ours(args):
         return e0.elapsed_time(e1) / steps
 
     for i in range(args.warmup):
-        e2e_step(i)
+        step(i)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = reduce_max(e2e_time(args.steps), world, device)
+    e2e_ms = reduce_max(timed(args.steps), world, device)
+    # what came back is the step's output: the same bits as the kernel-only graph
+    same = all(torch.equal(out_host[j].view(torch.int16), m.batches[0].out.cpu().view(torch.int16))
+               for j in range(2)) if b0.out.dtype == torch.bfloat16 else True
+    graphs.clear()
+    return {"ms_per_step": e2e_ms, "h2d_bytes_per_step": off, "d2h_bytes_per_step": d2h, "output_matches": same}
 
-    errs = [pa.workspace_error(b.workspace) for b in batches]
-    if any(errs):
-        raise SystemExit(f"kernel error word set: {errs}")
-    g_step.clear()  # release the graphs before the process group
-    g_attend.clear()
+
+PER_CONFIG = ("prefix_bf16", "fp8_long", "mixed_prefill_bs16", "mixed_prefill_bs32")
+
+
+def bench_ours(args):
+    world, rank, local = dist_setup(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import paged_kv_cache_452_b200 as pa  # noqa: F401  (fails loudly without libpa.so)
+    from paged_kv_cache_452_b200 import runner
+
+    peaks, src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0)))
+
+    wl = W.make(args.workload, "full")
+    if args.max_seqs:
+        wl = W.first_seqs(wl, args.max_seqs)
+    m = Measured(wl, device, args, world, rank, local)
+    stream = torch.cuda.current_stream()
+    # the same step issued launch by launch from Python (no graph)
+    eager_ms = reduce_max(_time(lambda i: runner.step(m.batches[i & 1]), args.steps, stream), world, device)
+    e2e = e2e_measure(m, device, args, world)
+    m.check()
+    head = m.summary(world, hbm, tc_peak)
+    cpu = cpu_baseline(wl, args.ref_budget) if (rank == 0 and not args.no_cpu_baseline) else None
+    m.release()
+
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name == wl.name:
+                continue
+            wl_c = W.make(name, "full")
+            mc = Measured(wl_c, device, args, world, rank, local)
+            mc.check()
+            per_config[name] = mc.summary(world, hbm, tc_peak)
+            mc.release()
+            if rank == 0 and not args.no_cpu_baseline:
+                per_config[name]["cpu_baseline"] = cpu_baseline(wl_c, min(args.ref_budget, 4.0))
 
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
         return
-    peaks, src = measured_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    achieved = alg_bytes / (attend_ms * 1e-3) / 1e9
+    achieved = m.alg_bytes / (m.attend_ms * 1e-3) / 1e9
+    kernel = "decode_tc_kernel (pa_decode)" if int(wl.q_lens.max()) == 1 else \
+        "decode_tc_kernel + prefill_umma_kernel (pa_decode_chunked_prefill)"
     line = {
-        "metric": METRIC, "value": job_throughput(world, alg_bytes, ms), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "metric": METRIC, "value": job_throughput(world, m.alg_bytes, m.ms), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.kv_dtype if wl.kv_dtype != "e4m3" else "fp8_e4m3",
         "data": "synthetic",
         "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": wl.block_size,
-                   "context_tokens": int((wl.context_lens + wl.q_lens).sum()), "kv_bytes": kv_bytes,
-                   "algorithmic_bytes": alg_bytes, "parallelism": f"replicas x{world}",
+                   "context_tokens": head["context_tokens"], "kv_bytes": m.kv_bytes,
+                   "algorithmic_bytes": m.alg_bytes, "parallelism": f"replicas x{world}",
                    "step": "pa_cache_write + pa_decode, replayed as a CUDA graph",
                    "l2": "2 pool copies used alternately, each larger than L2"},
-        "decode_tokens_per_s": world * wl.num_seqs / (ms * 1e-3),
-        "fraction_of_8tbs": alg_bytes / (ms * 1e-3) / 1e9 / 8000.0,
+        "decode_tokens_per_s": head["decode_tokens_per_s"],
+        "fraction_of_8tbs": m.alg_bytes / (m.ms * 1e-3) / 1e9 / 8000.0,
         "eager_ms_per_step": eager_ms,
-        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (pa_decode)",
+        "roofline": {"bound": "hbm", "kernel": kernel,
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src, "traffic": profiled_traffic(wl.name), "kernel_ms": attend_ms},
-        "e2e": {"value": job_throughput(world, alg_bytes, e2e_ms), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "pipelining": "uploads and downloads on their own streams, two input sets"},
+                     "peak_source": src, "traffic": profiled_traffic(wl.name), "kernel_ms": m.attend_ms},
+        "e2e": {"value": job_throughput(world, m.alg_bytes, e2e["ms_per_step"]), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                "ms_per_step": e2e["ms_per_step"], "output_matches": e2e["output_matches"],
+                "pipelining": "inputs uploaded as one packed copy on an upload stream, the step a CUDA graph "
+                              "of the public calls, output read back on a download stream; two input sets"},
         # pa_cache_write + pa_decode's decode kernel (+ its prefill kernel for prompt rows)
         "gpu_launches": (3 if int(wl.q_lens.max()) > 1 else 2) * args.steps,
-        "clocks": clocks,
+        "clocks": m.clocks,
     }
-    if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, args.ref_budget)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if per_config:
+        line["per_config"] = per_config
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -571,6 +767,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure only --workload, not the other full-size workloads")
+    ap.add_argument("--max-seqs", type=int, default=0,
+                    help="only the first N sequences of --workload (a smaller case of the same mix, "
+                         "for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

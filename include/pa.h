@@ -70,6 +70,16 @@ typedef struct {
   int32_t q_dtype;      /* pa_dtype of queries, new K/V and outputs: PA_F32 or PA_BF16 */
   float k_scale;        /* per-tensor scales of an e4m3 pool (stored = e4m3(x / scale)); */
   float v_scale;        /* ignored for fp32/bf16 pools */
+  /* Per-kv-head scales of an e4m3 pool: NULL, or a device array of
+   * num_kv_heads positive finite fp32 values (4-byte aligned, owned by the
+   * caller, read by the kernels): kv head h stores e4m3(x / scale[h]) and
+   * its codes dequantise to code * scale[h]; k_scale (v_scale) is then
+   * unused for K (V).  Ignored for fp32/bf16 pools.  The pages leave the
+   * granularity of an FP8 cache's scale open ("PagedAttention：KV cache
+   * 即虚拟内存（block manager & 碎片）", the num_gpu_blocks formula and the
+   * follow-up on a KV-bound step). */
+  const float* k_head_scales;
+  const float* v_head_scales;
 } pa_cache_desc;
 
 /* Message for the last failing call on this thread ("" if none). */
@@ -100,6 +110,27 @@ int pa_cache_write(const pa_cache_desc* desc, const void* k_new, const void* v_n
                    const int64_t* slot_mapping, int32_t num_tokens, void* k_cache, void* v_cache,
                    void* stream);
 
+/* pa_decode_fused: pa_cache_write of each sequence's new token and
+ * pa_decode, in one launch (the write of "write(blocks[-1], kv)" in the
+ * block-table snippet on "49 vLLM / PagedAttention", followed by the step's
+ * attention).  Sequence s's new token sits at position p = seq_lens[s] - 1
+ * (seq_lens counts it, as for pa_decode); its rows k_new[s], v_new[s] are
+ * stored at p's slot, block_tables[s][p / block_size] * block_size +
+ * p % block_size, as exactly the bytes pa_cache_write stores (e4m3
+ * quantisation included), and the attention over keys 0 .. p uses them.
+ * The result (pool bytes and out) equals pa_cache_write followed by
+ * pa_decode; only the tensor-core decode path is fused (bf16 queries, a bf16
+ * or e4m3 pool, GQA group 2..8; head_dim 64/128 for bf16, 128 for e4m3):
+ * other descs give PA_ERR_UNSUPPORTED.
+ *   k_new, v_new   device, [num_seqs][num_kv_heads][head_dim], bf16
+ *   k_cache, v_cache  device pools, written at each new token's slot
+ *   other arguments and the workspace as for pa_decode (a sequence with
+ *   seq_lens[s] == 0 writes nothing and gives a zero row). */
+int pa_decode_fused(const pa_cache_desc* desc, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                    void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* seq_lens, int32_t num_seqs, float scale, void* out, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
 /* pa_copy_blocks: the device half of copy-on-write ("PagedAttention：KV
  * cache 即虚拟内存（block manager & 碎片）", 深入原理, 共享 → prefix caching: a
  * fork that diverges inside a shared block triggers a copy).  For i < n, K
@@ -122,6 +153,10 @@ size_t pa_decode_workspace_size(const pa_cache_desc* desc, int32_t num_seqs);
  * row (row s of q) at position seq_lens[s] - 1 and attends its keys
  * 0 .. seq_lens[s] - 1, gathered through block_tables[s]; seq_lens counts
  * the token written this step.  out[s][h][:] = softmax(scale * q K^T) V.
+ * The block table plays the page table's part ("49 vLLM / PagedAttention",
+ * «Идея и механизм»); the result is the one dense attention gives over the
+ * same keys ("PagedAttention：KV cache 即虚拟内存（block manager & 碎片）",
+ * the follow-up "分页改变输出或加速 kernel 吗？").
  *   q           device, [num_seqs][num_q_heads][head_dim], q_dtype
  *   block_tables device, int32 [num_seqs][max_blocks_per_seq]
  *   seq_lens    device, int32 [num_seqs]; 0 gives a zero output row
@@ -135,7 +170,17 @@ size_t pa_decode_workspace_size(const pa_cache_desc* desc, int32_t num_seqs);
  *               3 = a sequence longer than its table row (clamped).  Read it
  *               after the stream synchronises; after any error, zero the
  *               whole workspace again.  Calls sharing a workspace must not
- *               overlap on the GPU.
+ *               overlap on the GPU.  Bytes 4..7 are a fault-injection word
+ *               for tests, zero in normal use: set to 1, the later pieces of
+ *               a context split over several warps do not report in, so the
+ *               merging warp's bounded wait runs out (after 1 ms) and sets
+ *               error word 1 without any fault; that call's output is wrong.
+ * Forward progress: the split-K merge waits for pieces held by other CTAs
+ * of the same launch, so the launch is sized to be resident all at once
+ * (the CTAs per SM the runtime reports, times the SMs).  Do not run two
+ * pa_decode calls at the same time on one GPU (separate streams without an
+ * ordering between them): each could hold SMs the other's waiting pieces
+ * need, and both would end at the 2 s bound with error word 1.
  * Long contexts are split over many CTAs (split-K over blocks) and merged
  * with a log-sum-exp combine; the split points depend only on seq_lens and
  * the device, so a result does not depend on where the blocks sit. */
@@ -156,11 +201,70 @@ int pa_decode(const pa_cache_desc* desc, const void* q, const void* k_cache, con
  * The first call on a device looks up the area's device address (with that
  * device current); make that first call before any stream capture.  Every
  * call clears the area's error word and arrival counters on `stream` first,
- * so in-kernel error reports are not kept between calls.  All calls share
+ * so the in-kernel reports that pa_decode leaves in its workspace's error
+ * word are neither kept between calls nor readable by the caller: a call
+ * whose kernel met an out-of-pool table entry or a timed-out wait still
+ * returns PA_OK (use pa_decode where those reports are needed).  Argument
+ * checks are pa_decode's, made before anything is enqueued.  All calls share
  * the one area: calls that overlap on the GPU race.  Allocates nothing. */
 int pa_decode_static(const pa_cache_desc* desc, const void* q, const void* k_cache, const void* v_cache,
                      const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                      int32_t num_seqs, float scale, void* out, void* stream);
+
+/* ---- shared prefixes ------------------------------------------------------
+ * Sequences admitted with prefix caching share the physical blocks of a
+ * common prefix (ref_cnt > 1; "49 vLLM / PagedAttention", Почему это важно;
+ * "PagedAttention：KV cache 即虚拟内存（block manager & 碎片）", 深入原理,
+ * 共享 → prefix caching).  pa_decode reads those blocks once per sequence;
+ * pa_decode_prefix attends each shared prefix once for all its sequences,
+ * as one dense contraction (every member's query rows against the prefix's
+ * keys) on the tensor cores, and merges that partial result with each
+ * sequence's own suffix by a log-sum-exp combine. */
+
+/* pa_prefix_groups (host): the shared prefixes of a decode batch, from its
+ * block tables.  Sequences whose rows start with the same physical block form
+ * a group when there are two or more; the group's prefix is the longest run
+ * of leading table entries all members have in common, cut so that every
+ * member keeps at least its last token (position seq_lens[s] - 1) outside
+ * it.  Groups with an empty prefix are dropped.
+ *   block_tables  host int32 [num_seqs][max_blocks_per_seq]; seq_lens host
+ *                 int32 [num_seqs] (as for pa_decode)
+ *   outputs (host, caller-allocated): prefix_start [num_seqs + 1] and
+ *   prefix_members [num_seqs] (CSR: prefix p's sequences are
+ *   prefix_members[prefix_start[p] .. prefix_start[p+1] - 1], increasing),
+ *   prefix_blocks [num_seqs] (blocks in prefix p), seq_prefix / seq_slot
+ *   [num_seqs] (sequence s's prefix and its index in prefix_members, or -1),
+ *   *num_prefixes, *num_members. */
+int pa_prefix_groups(const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                     int32_t num_seqs, int32_t block_size, int32_t* prefix_start, int32_t* prefix_members,
+                     int32_t* prefix_blocks, int32_t* seq_prefix, int32_t* seq_slot, int32_t* num_prefixes,
+                     int32_t* num_members);
+
+/* Scratch bytes pa_decode_prefix needs: pa_decode's plus the prefixes'
+ * partial results (num_members sequences, prefixes of up to
+ * max_prefix_blocks blocks). */
+size_t pa_decode_prefix_workspace_size(const pa_cache_desc* desc, int32_t num_seqs, int32_t num_members,
+                                       int32_t max_prefix_blocks);
+
+/* pa_decode_prefix: pa_decode's result for a batch with shared prefixes
+ * described as pa_prefix_groups gives them (device copies of its outputs):
+ *   prefix_start [num_prefixes + 1], prefix_members [num_members],
+ *   prefix_blocks [num_prefixes], seq_prefix [num_seqs], seq_slot [num_seqs]
+ *   device int32; max_prefix_blocks (host) >= every prefix_blocks[p].
+ * Every member's table row must hold the prefix's blocks in its first
+ * prefix_blocks[p] entries and its context must extend past them.  A bf16
+ * pool with bf16 queries, a GQA group of 2..8 and head_dim 64/128 runs the
+ * prefixes on a tcgen05 kernel, then the suffixes on the decode kernel,
+ * which folds each prefix partial in; other descs (and num_prefixes == 0)
+ * run pa_decode.  The workspace is as for pa_decode, sized by
+ * pa_decode_prefix_workspace_size; error word 4 = a context that does not
+ * extend past its prefix (that row is zero). */
+int pa_decode_prefix(const pa_cache_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                     int32_t num_seqs, const int32_t* prefix_start, const int32_t* prefix_members,
+                     const int32_t* prefix_blocks, const int32_t* seq_prefix, const int32_t* seq_slot,
+                     int32_t num_prefixes, int32_t num_members, int32_t max_prefix_blocks, float scale, void* out,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Scratch bytes pa_decode_chunked_prefill needs. */
 size_t pa_prefill_workspace_size(const pa_cache_desc* desc, int32_t num_seqs, int32_t num_tokens);

@@ -2,8 +2,8 @@
 
 This module draws numbers and nothing else: sequence lengths, the pool's
 initial free-list order, token ids for prefix hashing, N(0,1) query/key/value
-values cast to the input dtype, and per-tensor FP8 scales from the drawn
-values' absolute maximum.  It holds none of the method's arithmetic (no block
+values cast to the input dtype, and FP8 scales (per tensor or per kv head)
+from the drawn values' absolute maximum.  It holds none of the method's arithmetic (no block
 tables, slots, cache writes or attention); the oracle and the CUDA path each
 derive those from these same arrays.
 
@@ -68,10 +68,16 @@ class Workload:
     q_lens: np.ndarray  # int64 [S]: tokens added this step (1 = decode row)
     free_order: np.ndarray  # int32 [num_blocks]: initial free-list order
     prefix_len: int = 0
-    sharing: Optional[np.ndarray] = None  # bool [S]
+    sharing: Optional[np.ndarray] = None  # bool [S]: sequences sharing the one prefix
+    # several prefixes (tests): int [S], the prefix group of each sequence or
+    # -1; group g's prefix_len tokens are drawn from their own streams
+    prefix_group: Optional[np.ndarray] = None
     vocab: int = 32000
-    k_scale: float = 1.0
+    k_scale: float = 1.0  # e4m3 pools: one fp32 scale, or an array of one per kv head
     v_scale: float = 1.0
+    # how an e4m3 pool's scales are set: "tensor" (amax / 448 over every
+    # drawn value), "head" (amax / 448 per kv head) or "fixed" (as given)
+    scale_mode: str = "tensor"
     _fixed: Optional[dict] = field(default=None, repr=False)
     _amax: Optional[dict] = field(default=None, repr=False)
 
@@ -91,15 +97,25 @@ class Workload:
     # ---- draws ---------------------------------------------------------------
     def token_ids(self, s: int) -> Optional[np.ndarray]:
         """Token ids of the cached context of sequence s (None: no hashing)."""
-        if self.sharing is None:
+        if self.sharing is None and self.prefix_group is None:
             return None
         n = int(self.context_lens[s])
         own = rng(self.seed_key, s, S_TOKENS).integers(0, self.vocab, size=n, dtype=np.int64)
-        if self.sharing[s]:
-            pre = rng(self.seed_key, GLOBAL, S_TOKENS).integers(0, self.vocab, size=self.prefix_len,
-                                                                dtype=np.int64)
+        src = self._prefix_stream(s)
+        if src is not None:
+            pre = rng(self.seed_key, src, S_TOKENS).integers(0, self.vocab, size=self.prefix_len,
+                                                             dtype=np.int64)
             own[: self.prefix_len] = pre
         return own.astype(np.int32)
+
+    def _prefix_stream(self, s: int) -> Optional[int]:
+        """Sequence index of the streams sequence s's shared prefix is drawn
+        from (None: no shared prefix)."""
+        if self.sharing is not None and self.sharing[s]:
+            return GLOBAL
+        if self.prefix_group is not None and self.prefix_group[s] >= 0:
+            return GLOBAL - 1 - int(self.prefix_group[s])
+        return None
 
     def _normal(self, seq: int, stream: int, rows: int, heads: int) -> np.ndarray:
         return rng(self.seed_key, seq, stream).standard_normal((rows, heads, self.head_dim),
@@ -113,10 +129,11 @@ class Workload:
         n = int(self.context_lens[s])
         k = self._normal(s, S_K, n, self.num_kv_heads)
         v = self._normal(s, S_V, n, self.num_kv_heads)
-        if self.sharing is not None and self.sharing[s]:
+        src = self._prefix_stream(s)
+        if src is not None:
             p = self.prefix_len
-            k[:p] = self._normal(GLOBAL, S_K, p, self.num_kv_heads)
-            v[:p] = self._normal(GLOBAL, S_V, p, self.num_kv_heads)
+            k[:p] = self._normal(src, S_K, p, self.num_kv_heads)
+            v[:p] = self._normal(src, S_V, p, self.num_kv_heads)
         return k, v
 
     def prior_kv(self, s: int):
@@ -126,8 +143,7 @@ class Workload:
         k, v = _cast(k, self.q_dtype), _cast(v, self.q_dtype)
         if self._amax is None:
             self._amax = {}
-        self._amax[s] = (float(k.abs().max()) if k.numel() else 0.0,
-                         float(v.abs().max()) if v.numel() else 0.0)
+        self._amax[s] = (_head_amax(k, self.num_kv_heads), _head_amax(v, self.num_kv_heads))
         return k, v
 
     def new_kv(self):
@@ -145,27 +161,45 @@ class Workload:
             return _cast(self._fixed["q"], self.q_dtype)
         return _cast(self._normal(GLOBAL, S_Q, self.num_new_tokens, self.num_q_heads), self.q_dtype)
 
-    def set_fp8_scales(self, amax_k: float, amax_v: float):
-        """Per-tensor scales = amax / 448 (fp32), so the largest drawn value
-        maps onto the largest finite e4m3 value."""
-        self.k_scale = float(np.float32(amax_k) / np.float32(FP8_MAX))
-        self.v_scale = float(np.float32(amax_v) / np.float32(FP8_MAX))
+    def set_fp8_scales(self, amax_k, amax_v):
+        """Scales = amax / 448 (fp32), so the largest drawn value maps onto
+        the largest finite e4m3 value: one number each, or (arrays of amax)
+        one per kv head."""
+        def sc(a):
+            a = np.asarray(a, dtype=np.float32)
+            q = (a / np.float32(FP8_MAX)).astype(np.float32)
+            return float(q) if q.ndim == 0 else q
+        self.k_scale = sc(amax_k)
+        self.v_scale = sc(amax_v)
 
     def fp8_scales_from_draws(self):
         """amax over every K (V) value this workload draws, prior and new, in
-        the input dtype; sets and returns (k_scale, v_scale)."""
-        ak = av = 0.0
+        the input dtype (per kv head when scale_mode is "head"); sets and
+        returns (k_scale, v_scale).  scale_mode "fixed" keeps the given ones."""
+        if self.scale_mode == "fixed":
+            return self.k_scale, self.v_scale
+        ak = np.zeros(self.num_kv_heads, dtype=np.float32)
+        av = np.zeros(self.num_kv_heads, dtype=np.float32)
         for s in range(self.num_seqs):
             if self._amax is None or s not in self._amax:
                 self.prior_kv(s)
-            ak = max(ak, self._amax[s][0])
-            av = max(av, self._amax[s][1])
+            ak = np.maximum(ak, self._amax[s][0])
+            av = np.maximum(av, self._amax[s][1])
         k, v = self.new_kv()
-        if k.numel():
-            ak = max(ak, float(k.abs().max()))
-            av = max(av, float(v.abs().max()))
-        self.set_fp8_scales(ak, av)
+        ak = np.maximum(ak, _head_amax(k, self.num_kv_heads))
+        av = np.maximum(av, _head_amax(v, self.num_kv_heads))
+        if self.scale_mode == "head":
+            self.set_fp8_scales(ak, av)
+        else:
+            self.set_fp8_scales(ak.max(), av.max())
         return self.k_scale, self.v_scale
+
+
+def _head_amax(x: torch.Tensor, heads: int) -> np.ndarray:
+    """Largest |value| per kv head of a [rows][heads][head_dim] tensor."""
+    if x.numel() == 0:
+        return np.zeros(heads, dtype=np.float32)
+    return x.abs().amax(dim=(0, 2)).float().numpy().astype(np.float32)
 
 
 def _pool_size(need_blocks: int) -> int:
@@ -257,12 +291,39 @@ def mixed_prefill(block_size: int = 16, size: str = "full") -> Workload:
 
 
 def custom(name, context_lens, q_lens=None, kv_dtype="bf16", q_dtype="bf16", num_q_heads=8,
-           num_kv_heads=2, head_dim=128, block_size=16, seed_key=900, num_blocks=None) -> Workload:
-    """Explicit shapes for edge-case tests."""
+           num_kv_heads=2, head_dim=128, block_size=16, seed_key=900, num_blocks=None,
+           scale_mode="tensor", k_scale=1.0, v_scale=1.0, prefix_len=0, prefix_group=None) -> Workload:
+    """Explicit shapes for edge-case tests.  e4m3 scales: scale_mode
+    "tensor" / "head" derive them from the draws; "fixed" takes k_scale and
+    v_scale as given (a number, or one per kv head).  prefix_group (one int
+    per sequence, -1 for none): sequences of group g begin with the same
+    prefix_len tokens (token ids and K/V), which the pool's prefix hashing
+    then shares."""
     ctx = np.asarray(context_lens, dtype=np.int64)
     ql = np.ones_like(ctx) if q_lens is None else np.asarray(q_lens, dtype=np.int64)
-    return _finish(name, seed_key, kv_dtype, q_dtype, num_q_heads, num_kv_heads, head_dim,
-                   block_size, ctx, ql, nb=num_blocks)
+    wl = _finish(name, seed_key, kv_dtype, q_dtype, num_q_heads, num_kv_heads, head_dim,
+                 block_size, ctx, ql, nb=num_blocks)
+    wl.scale_mode = scale_mode
+    if prefix_group is not None:
+        wl.prefix_group = np.asarray(prefix_group, dtype=np.int64)
+        wl.prefix_len = int(prefix_len)
+        assert all(int(c) >= prefix_len for c, g in zip(ctx, wl.prefix_group) if g >= 0)
+    if scale_mode == "fixed":
+        wl.k_scale = k_scale if np.ndim(k_scale) == 0 else np.asarray(k_scale, dtype=np.float32)
+        wl.v_scale = v_scale if np.ndim(v_scale) == 0 else np.asarray(v_scale, dtype=np.float32)
+    return wl
+
+
+def first_seqs(wl: Workload, n: int) -> Workload:
+    """The first n sequences of a workload, with the same draws per sequence
+    and a pool sized (1.25x) and shuffled for them alone."""
+    n = min(n, wl.num_seqs)
+    sharing = None if wl.sharing is None else wl.sharing[:n].copy()
+    out = _finish(f"{wl.name}_first{n}", wl.seed_key, wl.kv_dtype, wl.q_dtype, wl.num_q_heads, wl.num_kv_heads,
+                  wl.head_dim, wl.block_size, wl.context_lens[:n], wl.q_lens[:n], prefix_len=wl.prefix_len,
+                  sharing=sharing)
+    out.scale_mode = wl.scale_mode
+    return out
 
 
 WORKLOADS = {

@@ -27,15 +27,21 @@ class CacheDesc(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
                 ("q_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
-                ("v_scale", ctypes.c_float)]
+                ("v_scale", ctypes.c_float), ("k_head_scales", ctypes.c_void_p),
+                ("v_head_scales", ctypes.c_void_p)]
 
     @classmethod
     def make(cls, num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, kv_dtype="bf16",
-             q_dtype="bf16", k_scale=1.0, v_scale=1.0):
+             q_dtype="bf16", k_scale=1.0, v_scale=1.0, k_head_scales=None, v_head_scales=None):
+        """k_head_scales / v_head_scales: optional device fp32 tensors
+        [num_kv_heads] (an e4m3 pool's per-kv-head scales); the desc keeps a
+        reference so they stay alive as long as it does."""
         kv = _CODES.get(kv_dtype, kv_dtype)
         q = _CODES.get(q_dtype, q_dtype)
-        return cls(num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, kv, q,
-                   float(k_scale), float(v_scale))
+        d = cls(num_blocks, block_size, num_kv_heads, num_q_heads, head_dim, kv, q,
+                float(k_scale), float(v_scale), _ptr(k_head_scales), _ptr(v_head_scales))
+        d._keep = (k_head_scales, v_head_scales)
+        return d
 
     @property
     def group(self):
@@ -138,6 +144,19 @@ def pa_decode(desc, q, k_cache, v_cache, block_tables, seq_lens, scale, out, wor
                            _stream(stream)), "pa_decode")
 
 
+def pa_decode_fused(desc, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale, out, workspace,
+                    stream=None):
+    """pa_cache_write of each sequence's new token (rows k_new[s], v_new[s],
+    at position seq_lens[s] - 1 through its block table) and pa_decode, in
+    one launch."""
+    s = int(seq_lens.shape[0])
+    _check(lib().pa_decode_fused(ctypes.byref(desc), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]), _ptr(seq_lens), s,
+                                 float(scale), _ptr(out), _ptr(workspace),
+                                 int(workspace.numel() * workspace.element_size()), _stream(stream)),
+           "pa_decode_fused")
+
+
 def pa_decode_static(desc, q, k_cache, v_cache, block_tables, seq_lens, scale, out, stream=None):
     """pa_decode without a workspace: the scratch is a fixed 8 MiB area built
     into the library, for callers that cannot allocate device memory."""
@@ -157,6 +176,56 @@ def pa_decode_chunked_prefill(desc, q, k_cache, v_cache, block_tables, query_sta
         int(max_q_len), float(scale), _ptr(out), _ptr(workspace),
         int(workspace.numel() * workspace.element_size()), _stream(stream)),
         "pa_decode_chunked_prefill")
+
+
+class PrefixGroups:
+    """Shared prefixes of a decode batch (pa_prefix_groups): CSR prefix_start
+    / prefix_members, prefix_blocks, and per sequence seq_prefix / seq_slot
+    (-1 outside any prefix), as int32 tensors on the host."""
+
+    def __init__(self, block_tables, seq_lens, block_size):
+        bt = block_tables.detach().cpu().contiguous().to(torch.int32)
+        sl = seq_lens.detach().cpu().contiguous().to(torch.int32)
+        n = int(sl.shape[0])
+        self.prefix_start = torch.zeros(n + 1, dtype=torch.int32)
+        self.prefix_members = torch.zeros(max(1, n), dtype=torch.int32)
+        self.prefix_blocks = torch.zeros(max(1, n), dtype=torch.int32)
+        self.seq_prefix = torch.zeros(max(1, n), dtype=torch.int32)
+        self.seq_slot = torch.zeros(max(1, n), dtype=torch.int32)
+        np_, nm = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().pa_prefix_groups(_ptr(bt), int(bt.shape[1]), _ptr(sl), n, int(block_size),
+                                      _ptr(self.prefix_start), _ptr(self.prefix_members), _ptr(self.prefix_blocks),
+                                      _ptr(self.seq_prefix), _ptr(self.seq_slot), ctypes.byref(np_),
+                                      ctypes.byref(nm)), "pa_prefix_groups")
+        self.num_prefixes, self.num_members = np_.value, nm.value
+        self.max_prefix_blocks = int(self.prefix_blocks[:self.num_prefixes].max()) if self.num_prefixes else 0
+
+    def to(self, device):
+        """The arrays pa_decode_prefix reads, on `device` (a dict)."""
+        return {k: getattr(self, k).to(device) for k in
+                ("prefix_start", "prefix_members", "prefix_blocks", "seq_prefix", "seq_slot")}
+
+
+def pa_decode_prefix_workspace_size(desc, num_seqs, num_members, max_prefix_blocks) -> int:
+    n = int(lib().pa_decode_prefix_workspace_size(ctypes.byref(desc), int(num_seqs), int(num_members),
+                                                  int(max_prefix_blocks)))
+    if n == 0:
+        raise PaError(1, "pa_decode_prefix_workspace_size: " + lib().pa_last_error().decode())
+    return n
+
+
+def pa_decode_prefix(desc, q, k_cache, v_cache, block_tables, seq_lens, groups, dev_groups, scale, out,
+                     workspace, stream=None):
+    """pa_decode with each shared prefix attended once for all its sequences
+    (groups: a PrefixGroups; dev_groups: its arrays on the device)."""
+    s = int(seq_lens.shape[0])
+    g = dev_groups
+    _check(lib().pa_decode_prefix(
+        ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
+        _ptr(seq_lens), s, _ptr(g["prefix_start"]), _ptr(g["prefix_members"]), _ptr(g["prefix_blocks"]),
+        _ptr(g["seq_prefix"]), _ptr(g["seq_slot"]), int(groups.num_prefixes), int(groups.num_members),
+        int(groups.max_prefix_blocks), float(scale), _ptr(out), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _stream(stream)), "pa_decode_prefix")
 
 
 def default_scale(head_dim):

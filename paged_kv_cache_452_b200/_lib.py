@@ -19,7 +19,12 @@ SIGNATURES = {
     "pa_decode_workspace_size": (_SZ, [_P, _I32]),
     "pa_decode": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P, _SZ, _P]),
     "pa_decode_static": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P]),
+    "pa_decode_fused": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _F, _P, _P, _SZ, _P]),
     "pa_prefill_workspace_size": (_SZ, [_P, _I32, _I32]),
+    "pa_prefix_groups": (ctypes.c_int, [_P, _I32, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
+    "pa_decode_prefix_workspace_size": (_SZ, [_P, _I32, _I32, _I32]),
+    "pa_decode_prefix": (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P, _P, _P, _P, _I32, _I32, _I32,
+                                        _F, _P, _P, _SZ, _P]),
     "pa_decode_chunked_prefill": (ctypes.c_int,
                                   [_P, _P, _P, _P, _P, _I32, _P, _P, _I32, _I32, _I32, _F, _P, _P, _SZ, _P]),
     "pa_pool_create": (ctypes.c_int, [_I32, _I32, _P, _P]),

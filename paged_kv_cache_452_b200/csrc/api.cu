@@ -51,9 +51,15 @@ int check_desc(const pa_cache_desc* d, const char* who) {
     return fail(PA_ERR_UNSUPPORTED, "%s: block_size %d (built: 16, 32)", who, d->block_size);
   if (d->head_dim != 64 && d->head_dim != 128)
     return fail(PA_ERR_UNSUPPORTED, "%s: head_dim %d (built: 64, 128)", who, d->head_dim);
-  if (d->kv_dtype == kFP8 && !(std::isfinite(d->k_scale) && std::isfinite(d->v_scale) && d->k_scale > 0.f &&
-                               d->v_scale > 0.f))
-    return fail(PA_ERR_INVALID_ARG, "%s: e4m3 cache needs positive finite k_scale/v_scale", who);
+  if (d->kv_dtype == kFP8) {
+    // per-tensor scales must be usable wherever per-head ones are not given
+    if (!d->k_head_scales && !(std::isfinite(d->k_scale) && d->k_scale > 0.f))
+      return fail(PA_ERR_INVALID_ARG, "%s: e4m3 cache needs a positive finite k_scale or k_head_scales", who);
+    if (!d->v_head_scales && !(std::isfinite(d->v_scale) && d->v_scale > 0.f))
+      return fail(PA_ERR_INVALID_ARG, "%s: e4m3 cache needs a positive finite v_scale or v_head_scales", who);
+    if (!aligned(d->k_head_scales, 4) || !aligned(d->v_head_scales, 4))
+      return fail(PA_ERR_INVALID_ARG, "%s: misaligned head scales", who);
+  }
   if ((int64_t)d->num_blocks * d->num_kv_heads * d->block_size >= (int64_t)INT32_MAX)
     return fail(PA_ERR_UNSUPPORTED, "%s: pool rows exceed 2^31", who);
   return PA_OK;
@@ -138,6 +144,11 @@ int encode_kv_map(CUtensorMap* m, const void* base, int dt, const pa_cache_desc*
   cuuint64_t strides[1] = {(cuuint64_t)d->head_dim * eb};
   cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)d->block_size};
   cuuint32_t estr[2] = {1, 1};
+  // the row stride must step over a whole row and stay a multiple of 16
+  // bytes: a map whose strides overlap or shrink is refused before encoding
+  if (strides[0] < dims[0] * eb || strides[0] % 16 != 0)
+    return fail(PA_ERR_INVALID_ARG, "tensor map: row stride %llu bytes for %llu-byte rows",
+                (unsigned long long)strides[0], (unsigned long long)(dims[0] * eb));
   CUresult r = enc(m, dt == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -173,11 +184,46 @@ WsCarve carve(void* base, int num_seqs, int num_kv_heads, int group, int head_di
   return c;
 }
 
+// pa_decode_prefix runs the shared prefixes on the tcgen05 kernel: a bf16
+// pool and queries, a GQA group that the tensor-core decode takes and that
+// divides the kernel's 128 rows.
+bool prefix_path(const pa_cache_desc* d) {
+  return use_tc(d) && d->kv_dtype == kBF16 &&
+         prefill_umma_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, d->num_q_heads / d->num_kv_heads);
+}
+
+// Bytes of the prefix partials after pa_decode's own scratch.
+size_t prefix_partial_bytes(const pa_cache_desc* d, int32_t num_members, int32_t max_prefix_blocks, size_t* ml_bytes) {
+  const size_t chunks = ((size_t)max_prefix_blocks * d->block_size + kPrefixChunkKeys - 1) / kPrefixChunkKeys;
+  const size_t rows = chunks * (size_t)num_members * d->num_q_heads;
+  *ml_bytes = (rows * 2 * 4 + 255) / 256 * 256;
+  return *ml_bytes + rows * d->head_dim * 4;
+}
+
+// Shared prefixes of a pa_decode_prefix call, for the decode kernel.
+struct PrefixArgs {
+  const int32_t* seq_prefix;
+  const int32_t* seq_slot;
+  const int32_t* prefix_blocks;
+  const float* ml;
+  const float* o;
+  int32_t num_members;
+};
+
+// The new tokens' rows that pa_decode_fused writes in the decode launch.
+struct FusedWrite {
+  const void* k_new;
+  const void* v_new;
+  void* k_pool;
+  void* v_pool;
+};
+
 // Decode rows (q_len == 1) of a batch on the tensor-core path; qsl may be null.
 int run_decode_tc(const pa_cache_desc* d, const void* q, const void* k_cache, const void* v_cache,
                   const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, const int32_t* qsl,
                   int32_t num_seqs, int32_t num_rows, float scale, void* out, void* workspace,
-                  size_t workspace_bytes, cudaStream_t stream, const char* who) {
+                  size_t workspace_bytes, cudaStream_t stream, const char* who, const FusedWrite* fw = nullptr,
+                  const PrefixArgs* pa = nullptr) {
   int sms = 0;
   int rc = num_sms(&sms);
   if (rc) return rc;
@@ -208,14 +254,35 @@ int run_decode_tc(const pa_cache_desc* d, const void* q, const void* k_cache, co
   p.group = group;
   const float log2e = 1.4426950408889634f;
   if (d->kv_dtype == kFP8) {
-    // f16 operands hold e4m3 values times 2^-8
-    p.scale_log2 = scale * log2e * d->k_scale * 256.f;
-    p.out_scale = d->v_scale * 256.f;
+    // f16 operands hold the stored e4m3 values; the dequantisation scales
+    // fold into the softmax scale and the output scale (per piece, when
+    // they are per kv head)
+    p.k_head = d->k_head_scales;
+    p.v_head = d->v_head_scales;
+    p.scale_log2 = scale * log2e * (p.k_head ? 1.f : d->k_scale);
+    p.out_scale = p.v_head ? 1.f : d->v_scale;
+    p.k_scale_w = d->k_scale;
+    p.v_scale_w = d->v_scale;
   } else {
     p.scale_log2 = scale * log2e;
     p.out_scale = 1.f;
   }
   p.ws = c.ws;
+  if (pa) {
+    p.pfx_of = pa->seq_prefix;
+    p.pfx_slot = pa->seq_slot;
+    p.pfx_blocks = pa->prefix_blocks;
+    p.pfx_ml = pa->ml;
+    p.pfx_o = pa->o;
+    p.pfx_members = pa->num_members;
+    p.pfx_chunk_blocks = kPrefixChunkKeys / d->block_size;
+  }
+  if (fw) {
+    p.k_new = static_cast<const uint8_t*>(fw->k_new);
+    p.v_new = static_cast<const uint8_t*>(fw->v_new);
+    p.k_pool = static_cast<uint8_t*>(fw->k_pool);
+    p.v_pool = static_cast<uint8_t*>(fw->v_pool);
+  }
   cudaError_t e = launch_decode_tc(p, tm_k, tm_v, d->kv_dtype, d->head_dim, d->block_size, sms, stream);
   if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "%s: shape not built for the tensor-core path", who);
   return cuda_status(e, who);
@@ -245,6 +312,10 @@ int run_simt(const pa_cache_desc* d, const void* q, const void* k_cache, const v
   p.scale = scale;
   p.k_scale = d->k_scale;
   p.v_scale = d->v_scale;
+  if (d->kv_dtype == kFP8) {
+    p.k_head = d->k_head_scales;
+    p.v_head = d->v_head_scales;
+  }
   p.only_multi_row = only_multi_row;
   cudaError_t e = launch_attn_simt(p, d->q_dtype, d->kv_dtype, stream);
   if (e == cudaErrorNotSupported)
@@ -253,6 +324,26 @@ int run_simt(const pa_cache_desc* d, const void* q, const void* k_cache, const v
 }
 
 }  // namespace
+
+int check_attn_args(const pa_cache_desc* d, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t num_seqs,
+                    void* out, void* workspace, const char* who) {
+  int rc = check_desc(d, who);
+  if (rc) return rc;
+  if (num_seqs < 0 || max_blocks < 0) return fail(PA_ERR_INVALID_ARG, "%s: negative size", who);
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out || !workspace)
+    return fail(PA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 256))
+    return fail(PA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
+  if (num_seqs > 16384) return fail(PA_ERR_UNSUPPORTED, "%s: more than 16384 sequences per call", who);
+  // (sequence, kv head, block) tiles are indexed with 32-bit integers
+  if ((int64_t)num_seqs * max_blocks * d->num_kv_heads >= (int64_t)INT32_MAX)
+    return fail(PA_ERR_UNSUPPORTED, "%s: num_seqs * max_blocks_per_seq * num_kv_heads reaches 2^31", who);
+  return PA_OK;
+}
+
 }  // namespace pa
 
 using namespace pa;
@@ -296,6 +387,10 @@ int pa_cache_write(const pa_cache_desc* d, const void* k_new, const void* v_new,
   p.num_slots = (int64_t)d->num_blocks * d->block_size;
   p.k_scale = d->k_scale;
   p.v_scale = d->v_scale;
+  if (d->kv_dtype == kFP8) {
+    p.k_head = d->k_head_scales;
+    p.v_head = d->v_head_scales;
+  }
   return cuda_status(launch_cache_write(p, d->q_dtype, d->kv_dtype, static_cast<cudaStream_t>(stream)),
                      "pa_cache_write");
 }
@@ -332,25 +427,6 @@ size_t pa_decode_workspace_size(const pa_cache_desc* d, int32_t num_seqs) {
   return decode_tc_workspace_bytes(num_seqs, d->num_kv_heads, d->num_q_heads / d->num_kv_heads, d->head_dim, sms);
 }
 
-static int check_attn_args(const pa_cache_desc* d, const void* q, const void* k_cache, const void* v_cache,
-                           const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens,
-                           int32_t num_seqs, void* out, void* workspace, const char* who) {
-  int rc = check_desc(d, who);
-  if (rc) return rc;
-  if (num_seqs < 0 || max_blocks < 0) return fail(PA_ERR_INVALID_ARG, "%s: negative size", who);
-  if (num_seqs == 0) return PA_OK;
-  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out || !workspace)
-    return fail(PA_ERR_INVALID_ARG, "%s: NULL pointer", who);
-  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 256))
-    return fail(PA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
-  if (num_seqs > 16384) return fail(PA_ERR_UNSUPPORTED, "%s: more than 16384 sequences per call", who);
-  // (sequence, kv head, block) tiles are indexed with 32-bit integers
-  if ((int64_t)num_seqs * max_blocks * d->num_kv_heads >= (int64_t)INT32_MAX)
-    return fail(PA_ERR_UNSUPPORTED, "%s: num_seqs * max_blocks_per_seq * num_kv_heads reaches 2^31", who);
-  return PA_OK;
-}
-
 int pa_decode(const pa_cache_desc* d, const void* q, const void* k_cache, const void* v_cache,
               const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
               float scale, void* out, void* workspace, size_t workspace_bytes, void* stream) {
@@ -365,6 +441,100 @@ int pa_decode(const pa_cache_desc* d, const void* q, const void* k_cache, const 
   if (workspace_bytes < 256) return fail(PA_ERR_INVALID_ARG, "pa_decode: workspace < 256 bytes");
   return run_simt(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, nullptr, num_seqs, num_seqs,
                   0, scale, out, workspace, st, "pa_decode");
+}
+
+int pa_decode_fused(const pa_cache_desc* d, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                    void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                    int32_t num_seqs, float scale, void* out, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  clear_error();
+  const char* who = "pa_decode_fused";
+  int rc = check_attn_args(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, out,
+                           workspace, who);
+  if (rc || num_seqs == 0) return rc;
+  if (!k_new || !v_new) return fail(PA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return fail(PA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
+  if (!use_tc(d))
+    return fail(PA_ERR_UNSUPPORTED, "%s: the write is fused only into the tensor-core decode (bf16 queries, "
+                "GQA group 2..8); use pa_cache_write + pa_decode", who);
+  const FusedWrite fw{k_new, v_new, k_cache, v_cache};
+  return run_decode_tc(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, nullptr, num_seqs, num_seqs,
+                       scale, out, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), who, &fw);
+}
+
+size_t pa_decode_prefix_workspace_size(const pa_cache_desc* d, int32_t num_seqs, int32_t num_members,
+                                       int32_t max_prefix_blocks) {
+  const size_t base = pa_decode_workspace_size(d, num_seqs);
+  if (base == 0 || num_members < 0 || max_prefix_blocks < 0) return 0;
+  if (!prefix_path(d)) return base;
+  size_t ml_bytes = 0;
+  return base + prefix_partial_bytes(d, num_members, max_prefix_blocks, &ml_bytes);
+}
+
+int pa_decode_prefix(const pa_cache_desc* d, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                     int32_t num_seqs, const int32_t* prefix_start, const int32_t* prefix_members,
+                     const int32_t* prefix_blocks, const int32_t* seq_prefix, const int32_t* seq_slot,
+                     int32_t num_prefixes, int32_t num_members, int32_t max_prefix_blocks, float scale, void* out,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  clear_error();
+  const char* who = "pa_decode_prefix";
+  int rc = check_attn_args(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, out,
+                           workspace, who);
+  if (rc || num_seqs == 0) return rc;
+  if (num_prefixes < 0 || num_members < 0 || max_prefix_blocks < 0 || num_members > num_seqs ||
+      max_prefix_blocks > max_blocks_per_seq)
+    return fail(PA_ERR_INVALID_ARG, "%s: bad prefix sizes", who);
+  if (num_prefixes == 0 || !prefix_path(d))
+    return pa_decode(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, scale, out,
+                     workspace, workspace_bytes, stream);
+  if (!prefix_start || !prefix_members || !prefix_blocks || !seq_prefix || !seq_slot)
+    return fail(PA_ERR_INVALID_ARG, "%s: NULL prefix array", who);
+  if (!aligned(prefix_start, 4) || !aligned(prefix_members, 4) || !aligned(prefix_blocks, 4) ||
+      !aligned(seq_prefix, 4) || !aligned(seq_slot, 4))
+    return fail(PA_ERR_INVALID_ARG, "%s: misaligned prefix array", who);
+  const size_t base = pa_decode_workspace_size(d, num_seqs);
+  size_t ml_bytes = 0;
+  const size_t need = base + prefix_partial_bytes(d, num_members, max_prefix_blocks, &ml_bytes);
+  if (base == 0 || workspace_bytes < need)
+    return fail(PA_ERR_INVALID_ARG, "%s: workspace %zu < %zu bytes", who, workspace_bytes, need);
+  int sms = 0;
+  if ((rc = num_sms(&sms))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* pml = reinterpret_cast<float*>(ws + base);
+  float* po = reinterpret_cast<float*>(ws + base + ml_bytes);
+  // 1. every shared prefix once for all its members: chunk partials
+  CUtensorMap tm_k, tm_v;
+  if ((rc = make_kv_map(&tm_k, k_cache, d->kv_dtype, d))) return rc;
+  if ((rc = make_kv_map(&tm_v, v_cache, d->kv_dtype, d))) return rc;
+  PrefillParams pp = {};
+  pp.q = static_cast<const uint8_t*>(q);
+  pp.block_tables = block_tables;
+  pp.max_blocks = max_blocks_per_seq;
+  pp.rows.num_seqs = num_prefixes;
+  pp.num_q_heads = d->num_q_heads;
+  pp.num_kv_heads = d->num_kv_heads;
+  pp.group = d->num_q_heads / d->num_kv_heads;
+  pp.num_blocks = d->num_blocks;
+  pp.scale_log2 = scale * 1.4426950408889634f;
+  pp.err = static_cast<int32_t*>(workspace);
+  pp.pfx_start = prefix_start;
+  pp.pfx_members = prefix_members;
+  pp.pfx_blocks = prefix_blocks;
+  pp.num_members = num_members;
+  pp.chunk_keys = kPrefixChunkKeys;
+  pp.pfx_ml = pml;
+  pp.pfx_o = po;
+  cudaError_t e = launch_prefix_umma(pp, tm_k, tm_v, d->head_dim, d->block_size, sms, st);
+  if (e == cudaErrorNotSupported)
+    return pa_decode(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, scale, out,
+                     workspace, workspace_bytes, stream);
+  if ((rc = cuda_status(e, who))) return rc;
+  // 2. the suffixes on the decode kernel, folding each member's chunk partials
+  const PrefixArgs pa{seq_prefix, seq_slot, prefix_blocks, pml, po, num_members};
+  return run_decode_tc(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, nullptr, num_seqs,
+                       num_seqs, scale, out, workspace, base, st, who, nullptr, &pa);
 }
 
 size_t pa_prefill_workspace_size(const pa_cache_desc* d, int32_t num_seqs, int32_t num_tokens) {

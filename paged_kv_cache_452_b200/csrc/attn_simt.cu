@@ -23,10 +23,7 @@ __device__ __forceinline__ float load_kv(const uint8_t* base, int64_t idx) {
   } else if constexpr (KV == kBF16) {
     return dev::bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(base)[idx]);
   } else {
-    // e4m3 byte -> f16 bits of value * 2^-8 (exact, see pa_device.cuh) -> fp32
-    const uint32_t b = base[idx];
-    const uint16_t h = (uint16_t)(((b + (b & 0x80u)) << 7) & 0xFFFFu);
-    return __half2float(__ushort_as_half(h)) * 256.0f;
+    return dev::e4m3_to_f32(base[idx]);  // exact
   }
 }
 
@@ -69,6 +66,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
     pos = p.max_blocks * p.block_size - 1;
   }
   const int kvh = h / (hq / p.num_kv_heads);
+  const float ks = p.k_head ? __ldg(p.k_head + kvh) : p.k_scale;  // e4m3 dequantisation scales
+  const float vs = p.v_head ? __ldg(p.v_head + kvh) : p.v_scale;
   const int hkv = p.num_kv_heads, bs = p.block_size;
   const int64_t qo = ((int64_t)r * hq + h) * D;
   float qv[E], acc[E];
@@ -92,7 +91,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
     for (int e = 0; e < E; ++e) dot += qv[e] * load_kv<KV>(p.k_cache, kb + lane + 32 * e);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (KV == kFP8) dot *= p.k_scale;
+    if (KV == kFP8) dot *= ks;
     const float mn = fmaxf(m, dot);
     const float corr = expf(m - mn), pj = expf(dot - mn);
     l = l * corr + pj;
@@ -104,7 +103,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const SimtParams p) {
     }
     m = mn;
   }
-  const float inv = (pos >= 0 ? 1.f / l : 0.f) * (KV == kFP8 ? p.v_scale : 1.f);
+  const float inv = (pos >= 0 ? 1.f / l : 0.f) * (KV == kFP8 ? vs : 1.f);
 #pragma unroll
   for (int e = 0; e < E; ++e) store_out<QT>(p.out, qo + lane + 32 * e, pos >= 0 ? acc[e] * inv : 0.f);
 }

@@ -14,13 +14,6 @@
 namespace pa {
 namespace {
 
-__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
-  uint16_t r;
-  // cvt packs its first source operand into the upper byte
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 // IN: element type of k_new/v_new (float or __nv_bfloat16); TO_FP8: quantise.
 template <typename IN, bool TO_FP8>
 __global__ void __launch_bounds__(256) cache_write_kernel(CacheWriteParams p) {
@@ -51,7 +44,8 @@ __global__ void __launch_bounds__(256) cache_write_kernel(CacheWriteParams p) {
                 (((blk * p.num_kv_heads + h) * p.block_size + off) * p.head_dim + (int64_t)c * VEC);
       *reinterpret_cast<uint4*>(dst) = raw;
     } else {
-      const float scale = side ? p.v_scale : p.k_scale;
+      const float* head = side ? p.v_head : p.k_head;
+      const float scale = head ? __ldg(head + h) : (side ? p.v_scale : p.k_scale);
       float x[VEC];
       if constexpr (sizeof(IN) == 4) {
         x[0] = __uint_as_float(raw.x);
@@ -69,7 +63,7 @@ __global__ void __launch_bounds__(256) cache_write_kernel(CacheWriteParams p) {
       uint8_t q[VEC];
 #pragma unroll
       for (int i = 0; i < VEC; i += 2) {
-        const uint16_t pair = e4m3x2_from_f32(__fdiv_rn(x[i], scale), __fdiv_rn(x[i + 1], scale));
+        const uint16_t pair = dev::e4m3x2_from_f32(__fdiv_rn(x[i], scale), __fdiv_rn(x[i + 1], scale));
         q[i] = (uint8_t)(pair & 0xFF);
         q[i + 1] = (uint8_t)(pair >> 8);
       }

@@ -16,7 +16,12 @@
 // before any stream capture.  All calls share the array and it keeps the
 // previous call's contents: each call clears the parts that must start at
 // zero (the error word and the arrival counters), and calls that overlap on
-// the GPU race on it.  Nothing here allocates.
+// the GPU race on it.  Because the error word lives in that array and the
+// next call clears it, the in-kernel reports pa_decode leaves in its
+// workspace (a bounded wait that ran out, a table entry outside the pool, a
+// context longer than its table row) cannot be read by a caller of this
+// entry point; callers that need them use pa_decode.  Nothing here
+// allocates.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -58,24 +63,31 @@ extern "C" int pa_decode_static(const pa_cache_desc* desc, const void* q, const 
                                 const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                                 int32_t num_seqs, float scale, void* out, void* stream) {
   pa::clear_error();
-  if (!desc) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode_static: desc is NULL");
-  if (num_seqs < 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode_static: num_seqs < 0");
-  if (num_seqs == 0) return PA_OK;
+  const char* who = "pa_decode_static";
+  // every check pa_decode makes on its arguments, before anything is
+  // enqueued; the workspace pointer it checks is a host stand-in (the
+  // scratch's device address is looked up only once the call is accepted)
+  alignas(256) static unsigned char workspace_stand_in[1];
+  int rc = pa::check_attn_args(desc, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+                               out, workspace_stand_in, who);
+  if (rc || num_seqs == 0) return rc;
   const size_t need = pa_decode_workspace_size(desc, num_seqs);
   if (need == 0) return PA_ERR_INVALID_ARG;  // the size query already recorded why
   if (need > kStaticScratchBytes)
     return pa::fail(PA_ERR_UNSUPPORTED,
-                    "pa_decode_static: this batch needs %zu bytes of scratch, the static area holds %zu; "
+                    "%s: this batch needs %zu bytes of scratch, the static area holds %zu; "
                     "use pa_decode with a workspace",
-                    need, kStaticScratchBytes);
+                    who, need, kStaticScratchBytes);
   void* ws = nullptr;
-  int rc = scratch_address(&ws);
-  if (rc) return rc;
-  // the error word (256 bytes) and the arrival counters (4 bytes per
-  // sequence and kv head, padded to 256) must start at zero
-  const size_t zeroed = 256 + ((size_t)num_seqs * desc->num_kv_heads * 4 + 255) / 256 * 256;
+  if ((rc = scratch_address(&ws))) return rc;
+  // what must start at zero: the error word (256 bytes) and, on the
+  // tensor-core path, the arrival counters (4 bytes per sequence and kv head,
+  // padded to 256); the CUDA-core path's scratch is the error word alone.
+  // Never more than the batch's own scratch, which fits in the area.
+  size_t zeroed = 256 + ((size_t)num_seqs * desc->num_kv_heads * 4 + 255) / 256 * 256;
+  if (zeroed > need) zeroed = need;
   cudaError_t e = cudaMemsetAsync(ws, 0, zeroed, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_static: %s", cudaGetErrorString(e));
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "%s: %s", who, cudaGetErrorString(e));
   return pa_decode(desc, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, scale, out, ws,
                    kStaticScratchBytes, stream);
 }

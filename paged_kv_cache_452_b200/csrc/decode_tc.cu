@@ -33,9 +33,9 @@
 //    keys on the MMA's M side and the group's query rows on N (8, padded):
 //    S^T = K Q^T and O^T += V^T P^T with mma.sync m16n8k16 (fp32 accumulate),
 //    an online softmax per query column, and P^T moved into the B operand
-//    with movmatrix.  e4m3 K/V become f16 exactly (bit placement, see
-//    pa_device.cuh), and the 2^8 factor plus the per-tensor scales are folded
-//    into the softmax scale and the output scale.
+//    with movmatrix.  e4m3 K/V become f16 exactly (the hardware's paired
+//    e4m3 -> f16x2 conversion, two per four bytes), and the per-tensor
+//    scales are folded into the softmax scale and the output scale.
 #include <cuda_runtime.h>
 
 #include "pa_device.cuh"
@@ -74,7 +74,7 @@ struct Cfg {
 };
 
 struct SmemLayout {
-  uint32_t ring, bars, info, prefix, total;
+  uint32_t ring, bars, info, prefix, skip, total;
 };
 
 // A stage holds one tile's K and V and, when the tile opens a (sequence, kv
@@ -82,7 +82,9 @@ struct SmemLayout {
 // the next stage's tiles stay 1 KB aligned for the 128-byte swizzle).
 __host__ __device__ inline int q_area_bytes(int group, int d) { return (group * d * 2 + 1023) / 1024 * 1024; }
 
-__host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int num_seqs) {
+// pfx: shared prefixes are skipped, so each sequence's skipped block count
+// is kept next to the tile prefix
+__host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int num_seqs, bool pfx) {
   SmemLayout L;
   uint32_t off = 0;
   L.ring = off;
@@ -93,6 +95,8 @@ __host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int 
   off += (uint32_t)kWarps * nsw * 16;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
+  L.skip = off;
+  if (pfx) off += (uint32_t)num_seqs * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
   return L;
 }
@@ -114,6 +118,16 @@ __device__ __forceinline__ int find_seq(const int32_t* prefix, int S, int hkv, i
 // CTA owning tile x.
 __device__ __forceinline__ int range_start(int c, int T, int P) { return (int)((int64_t)c * T / P); }
 __device__ __forceinline__ int cta_of(int x, int T, int P) { return (int)((((int64_t)x + 1) * P - 1) / T); }
+
+// e4m3 tiles: thread (g, t) of an ldmatrix holds bytes 4t..4t+3 of a row,
+// converted as the pairs (4t, 4t+1) -> A columns 2t, 2t+1 and (4t+2, 4t+3)
+// -> A columns 2t+8, 2t+9.  For P V, whose A rows are d and whose columns
+// are keys, logical k j therefore reads key kperm(j); S^T = K Q^T puts key
+// kperm(r) on its A row r so that P^T, moved into the B operand, follows the
+// same order.
+__device__ __forceinline__ int kperm(int r) {
+  return r < 8 ? 4 * (r >> 1) + (r & 1) : 4 * ((r - 8) >> 1) + 2 + (r & 1);
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -139,6 +153,61 @@ __device__ __forceinline__ unsigned int load_acquire(const unsigned int* cnt) {
   return v;
 }
 
+// pa_decode_fused's write, by the warp that owns sequence s's last tile
+// (its stage `st` has landed): the new token's K and V rows for kv head h
+// (row `row` of k_new / v_new) go to offset `key` of the sequence's last
+// block (entry nb - 1 of its table row) in the pools, as the bytes
+// pa_cache_write stores, and into the stage.  A context clamped to its table row (error 3) or a last block
+// outside the pool (error 2, already flagged) writes nothing to the pool.
+template <class C>
+__device__ __forceinline__ void fused_write(const DecodeParams& p, uint8_t* st, int s, int h, int row, int len,
+                                            int key, int nb, int lane) {
+  constexpr int BS = C::KM * 16, D = C::DM * 16;
+  if (__ldg(p.rows.seq_lens + s) != len) return;  // clamped context: the token is not in the table row
+  const int hkv = p.num_kv_heads;
+  const int blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + (nb - 1));
+  const bool to_pool = blk >= 0 && blk < p.num_blocks;
+  const int64_t nrow = ((int64_t)row * hkv + h) * D * 2;  // bf16 new rows
+  if constexpr (!C::FP8) {
+    // lanes 0..15: 16-byte units of the K row, lanes 16..31: of the V row
+    const int side = lane >> 4, u = lane & 15;
+    if (u < C::NCH * 8) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>((side ? p.v_new : p.k_new) + nrow + u * 16));
+      const int c = u >> 3, uu = u & 7;
+      *reinterpret_cast<uint4*>(st + side * C::TILE + c * BS * 128 + key * 128 + ((uu ^ (key & 7)) << 4)) = x;
+      if (to_pool)
+        *reinterpret_cast<uint4*>((side ? p.v_pool : p.k_pool) + (((int64_t)blk * hkv + h) * BS + key) * C::ROW +
+                                  u * 16) = x;
+    }
+  } else {
+    // lane l quantises d = 4l .. 4l+3 of the K row and of the V row
+    const float ks = p.k_head ? __ldg(p.k_head + h) : p.k_scale_w;
+    const float vs = p.v_head ? __ldg(p.v_head + h) : p.v_scale_w;
+    const uint2 kx = __ldg(reinterpret_cast<const uint2*>(p.k_new + nrow + 8 * lane));
+    const uint2 vx = __ldg(reinterpret_cast<const uint2*>(p.v_new + nrow + 8 * lane));
+    const uint32_t k01 = dev::e4m3x2_from_f32(__fdiv_rn(dev::bf16_bits_to_f32(kx.x & 0xFFFFu), ks),
+                                              __fdiv_rn(dev::bf16_bits_to_f32(kx.x >> 16), ks));
+    const uint32_t k23 = dev::e4m3x2_from_f32(__fdiv_rn(dev::bf16_bits_to_f32(kx.y & 0xFFFFu), ks),
+                                              __fdiv_rn(dev::bf16_bits_to_f32(kx.y >> 16), ks));
+    const uint32_t v01 = dev::e4m3x2_from_f32(__fdiv_rn(dev::bf16_bits_to_f32(vx.x & 0xFFFFu), vs),
+                                              __fdiv_rn(dev::bf16_bits_to_f32(vx.x >> 16), vs));
+    const uint32_t v23 = dev::e4m3x2_from_f32(__fdiv_rn(dev::bf16_bits_to_f32(vx.y & 0xFFFFu), vs),
+                                              __fdiv_rn(dev::bf16_bits_to_f32(vx.y >> 16), vs));
+    const uint32_t kw = k01 | (k23 << 16);
+    // K: token-major 128-byte row, 128-byte swizzle in the stage
+    *reinterpret_cast<uint32_t*>(st + key * 128 + (((lane >> 2) ^ (key & 7)) << 4) + 4 * (lane & 3)) = kw;
+    // V: d-major [D][BS], one byte per d
+    const uint8_t vb[4] = {(uint8_t)(v01 & 0xFF), (uint8_t)(v01 >> 8), (uint8_t)(v23 & 0xFF), (uint8_t)(v23 >> 8)};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st[C::TILE + (4 * lane + i) * BS + key] = vb[i];
+    if (to_pool) {
+      *reinterpret_cast<uint32_t*>(p.k_pool + (((int64_t)blk * hkv + h) * BS + key) * C::ROW + 4 * lane) = kw;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p.v_pool[(((int64_t)blk * hkv + h) * D + 4 * lane + i) * BS + key] = vb[i];
+    }
+  }
+}
+
 template <int KV, int D, int BS>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -151,8 +220,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
   const int hkv = p.num_kv_heads, G = p.group, hq = p.num_q_heads;
   const int QA = q_area_bytes(G, D);
   const int STAGE = C::KVB + QA;  // bytes per ring stage
-  const SmemLayout L = smem_layout(STAGE, NSW, S);
+  const bool pfx = p.pfx_of != nullptr;
+  const SmemLayout L = smem_layout(STAGE, NSW, S, pfx);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L.prefix);
+  // blocks of the sequence's row that a shared prefix covers (pa_decode_prefix)
+  int32_t* skipv = reinterpret_cast<int32_t*>(smem + L.skip);
   __shared__ int32_t warp_tot[kWarps];
 
   const int tid = threadIdx.x;
@@ -173,6 +245,23 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     if (nb > p.max_blocks) {  // context longer than its table row: flag, clamp
       atomicCAS(p.ws.err, 0, 3);
       nb = p.max_blocks;
+    }
+    if (pfx) {
+      // a shared prefix's blocks are attended by the prefix kernel: only the
+      // suffix is tiled here; its last token must lie past the prefix
+      int skip = 0;
+      const int pf = nb > 0 ? p.pfx_of[s] : -1;
+      if (pf >= 0) {
+        skip = p.pfx_blocks[pf];
+        if ((int64_t)skip * BS > (int64_t)len - 1 || skip >= nb) {
+          atomicCAS(p.ws.err, 0, 4);  // flag; the row stays zero
+          skip = 0;
+          nb = 0;
+        } else {
+          nb -= skip;
+        }
+      }
+      skipv[s] = skip;
     }
     prefix[s] = nb;
   }
@@ -249,7 +338,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
       const int nb = prefix[s + 1] - prefix[s];
       const int local = t - hkv * prefix[s];
       d.h = local / nb;
-      const int i = local - d.h * nb;
+      const int skip = pfx ? skipv[s] : 0;
+      const int i = local - d.h * nb + skip;
       d.blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + i);
       if (d.blk < 0 || d.blk >= p.num_blocks) {  // bad table entry: flag, read block 0
         atomicCAS(p.ws.err, 0, 2);
@@ -257,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
       }
       if (i == 0 || t == wbeg) {
         d.row = p.rows.qsl ? __ldg(p.rows.qsl + s) : s;
-        d.len = min(__ldg(p.rows.seq_lens + s), nb * BS);
+        d.len = min(__ldg(p.rows.seq_lens + s), (nb + skip) * BS);
       }
     }
     return d;
@@ -305,6 +395,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
   };
   int issued = 0;
   dev::grid_dep_wait();  // the pool rows this step wrote are visible from here on
+  // Fault injection for tests (the workspace's second word, zero in normal
+  // use): the later pieces of a cut context skip their count-in, so the
+  // merging warp's wait runs out, after 1 ms instead of 2 s, and reports it.
+  const bool inject = *reinterpret_cast<volatile const int32_t*>(p.ws.err + 1) == 1;
   for (; issued < NSW && issued < nmine; ++issued) issue(issued);
   nxt = describe(32);  // the next batch, needed from warp-tile 32 on
 
@@ -325,7 +419,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     const int h = (t - seg0) / nb;
     const int a = seg0 + h * nb, b = a + nb;
     const int pe = min(b, wend);
+    const int skip = pfx ? skipv[s] : 0;  // tile a holds block `skip` of the row
     int row = 0, len = 0;
+    // this kv head's softmax and output scales (e4m3 per-head dequantisation)
+    const float sl2 = p.k_head ? p.scale_log2 * __ldg(p.k_head + h) : p.scale_log2;
+    const float osc = p.v_head ? p.out_scale * __ldg(p.v_head + h) : p.out_scale;
     uint32_t qf[C::KSTEPS][2];
 
     float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
@@ -350,22 +448,30 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
             qf[kk][1] = g < G ? *reinterpret_cast<const uint32_t*>(qs + (16 * kk + 2 * tq + 8) * 2) : 0u;
           }
         } else {
-          // d order inside a 16-wide k-step follows the e4m3 byte split:
-          // logical k (2t, 2t+1 | 2t+8, 2t+9) <-> d (4t, 4t+2 | 4t+1, 4t+3)
+          // d order inside a 16-wide k-step follows the e4m3 byte pairs
+          // (a thread's four bytes of a K row are d 4t..4t+3):
+          // logical k (2t, 2t+1 | 2t+8, 2t+9) <-> d (4t, 4t+1 | 4t+2, 4t+3)
 #pragma unroll
           for (int kk = 0; kk < C::KSTEPS; ++kk) {
             uint2 w = make_uint2(0u, 0u);
             if (g < G) w = *reinterpret_cast<const uint2*>(qs + (16 * kk + 4 * tq) * 2);
             const float q0 = dev::bf16_bits_to_f32(w.x & 0xFFFFu), q1 = dev::bf16_bits_to_f32(w.x >> 16);
             const float q2 = dev::bf16_bits_to_f32(w.y & 0xFFFFu), q3 = dev::bf16_bits_to_f32(w.y >> 16);
-            qf[kk][0] = dev::pack_f16(q0, q2);
-            qf[kk][1] = dev::pack_f16(q1, q3);
+            qf[kk][0] = dev::pack_f16(q0, q1);
+            qf[kk][1] = dev::pack_f16(q2, q3);
           }
         }
       }
       const uint32_t kbase = ring_u32 + stage * STAGE;
       const uint32_t vbase = kbase + C::TILE;
-      const int key0 = (tile - a) * BS;
+      const int key0 = (tile - a + skip) * BS;
+      if (p.k_new != nullptr && tile == b - 1) {
+        // pa_decode_fused: the sequence's last tile holds its new token at
+        // position len - 1; store the token's K/V rows into the pool and
+        // over the landed tile, so the attention below uses them
+        fused_write<C>(p, ring + (size_t)stage * STAGE, s, h, row, len, len - 1 - key0, skip + nb, lane);
+        __syncwarp();
+      }
       if (len - key0 < BS) {
         // Slots past the context hold whatever the pool last stored there
         // (possibly NaN/Inf bit patterns): their scores are masked to -inf,
@@ -402,10 +508,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
             else dev::mma_bf16(acc0, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
           }
         } else {
-          // A-row r holds key 2r (r < 8) or 2(r-8)+1, matching the key order
-          // of the d-major V operand after the byte split
+          // A-row r holds key kperm(r), the key order of the d-major V
+          // operand after the byte pairing (logical k j <-> key kperm(j))
           const int ar = (li & 1) * 8 + lr;
-          const int key = 16 * km + (ar < 8 ? 2 * ar : 2 * (ar - 8) + 1);
+          const int key = 16 * km + kperm(ar);
 #pragma unroll
           for (int uu = 0; uu < C::KSTEPS / 2; ++uu) {
             const int unit = 2 * uu + (li >> 1);
@@ -413,21 +519,21 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
             uint32_t w0, w1, w2, w3;
             dev::ldsm_x4(addr, w0, w1, w2, w3);
             uint32_t l0w, h0w, l1w, h1w, l2w, h2w, l3w, h3w;
-            dev::e4m3x4_to_f16x2x2(w0, l0w, h0w);
-            dev::e4m3x4_to_f16x2x2(w1, l1w, h1w);
-            dev::e4m3x4_to_f16x2x2(w2, l2w, h2w);
-            dev::e4m3x4_to_f16x2x2(w3, l3w, h3w);
+            dev::e4m3x4_to_f16x2(w0, l0w, h0w);
+            dev::e4m3x4_to_f16x2(w1, l1w, h1w);
+            dev::e4m3x4_to_f16x2(w2, l2w, h2w);
+            dev::e4m3x4_to_f16x2(w3, l3w, h3w);
             dev::mma_f16(acc0, l0w, l1w, h0w, h1w, qf[2 * uu][0], qf[2 * uu][1]);
             dev::mma_f16(acc1, l2w, l3w, h2w, h3w, qf[2 * uu + 1][0], qf[2 * uu + 1][1]);
           }
         }
         // rows of this thread: keys r0 (row g) and r1 (row g+8)
-        const int r0 = key0 + 16 * km + (C::FP8 ? 2 * g : g);
-        const int r1 = key0 + 16 * km + (C::FP8 ? 2 * g + 1 : g + 8);
-        sc[km][0] = r0 < len ? (acc0[0] + acc1[0]) * p.scale_log2 : -INFINITY;
-        sc[km][1] = r0 < len ? (acc0[1] + acc1[1]) * p.scale_log2 : -INFINITY;
-        sc[km][2] = r1 < len ? (acc0[2] + acc1[2]) * p.scale_log2 : -INFINITY;
-        sc[km][3] = r1 < len ? (acc0[3] + acc1[3]) * p.scale_log2 : -INFINITY;
+        const int r0 = key0 + 16 * km + (C::FP8 ? kperm(g) : g);
+        const int r1 = key0 + 16 * km + (C::FP8 ? kperm(g + 8) : g + 8);
+        sc[km][0] = r0 < len ? (acc0[0] + acc1[0]) * sl2 : -INFINITY;
+        sc[km][1] = r0 < len ? (acc0[1] + acc1[1]) * sl2 : -INFINITY;
+        sc[km][2] = r1 < len ? (acc0[2] + acc1[2]) * sl2 : -INFINITY;
+        sc[km][3] = r1 < len ? (acc0[3] + acc1[3]) * sl2 : -INFINITY;
       }
 
       // ---- online softmax per query column (columns 2tq, 2tq+1) ----
@@ -495,10 +601,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
             uint32_t w0, w1, w2, w3;
             dev::ldsm_x4(vbase + d * BS + km * 16, w0, w1, w2, w3);
             uint32_t l0w, h0w, l1w, h1w, l2w, h2w, l3w, h3w;
-            dev::e4m3x4_to_f16x2x2(w0, l0w, h0w);
-            dev::e4m3x4_to_f16x2x2(w1, l1w, h1w);
-            dev::e4m3x4_to_f16x2x2(w2, l2w, h2w);
-            dev::e4m3x4_to_f16x2x2(w3, l3w, h3w);
+            dev::e4m3x4_to_f16x2(w0, l0w, h0w);
+            dev::e4m3x4_to_f16x2(w1, l1w, h1w);
+            dev::e4m3x4_to_f16x2(w2, l2w, h2w);
+            dev::e4m3x4_to_f16x2(w3, l3w, h3w);
             dev::mma_f16(o[2 * mt2], l0w, l1w, h0w, h1w, pb0[km], pb1[km]);
             dev::mma_f16(o[2 * mt2 + 1], l2w, l3w, h2w, h3w, pb0[km], pb1[km]);
           }
@@ -525,23 +631,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
     const int64_t obase = ((int64_t)row * hq + (int64_t)h * G) * D;
-    if (t == a && pe == b) {
-      // the whole context is in this warp's range: write the output
-      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + obase;
-      const float i0 = p.out_scale / l0, i1 = p.out_scale / l1;
-#pragma unroll
-      for (int mt = 0; mt < C::DM; ++mt) {
-        const int d0 = 16 * mt + g;
-        if (c0 < G) {
-          out[c0 * D + d0] = __float2bfloat16_rn(o[mt][0] * i0);
-          out[c0 * D + d0 + 8] = __float2bfloat16_rn(o[mt][2] * i0);
-        }
-        if (c1 < G) {
-          out[c1 * D + d0] = __float2bfloat16_rn(o[mt][1] * i1);
-          out[c1 * D + d0 + 8] = __float2bfloat16_rn(o[mt][3] * i1);
-        }
-      }
-    } else if (t != a) {
+    if (t != a) {
       // a later piece of a sequence cut by warp ranges (it starts this
       // warp's range, so each warp has at most one): store the partial in
       // the warp's slot and count it in
@@ -570,38 +660,20 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
         }
       }
       __syncwarp();
-      if (lane == 0) count_in_release(p.ws.cnt + (int64_t)s * hkv + h);
+      if (lane == 0 && !inject) count_in_release(p.ws.cnt + (int64_t)s * hkv + h);
     } else {
-      // the sequence's first piece, cut by the end of this warp's range:
-      // this warp merges.  It finishes after the other pieces (they sit at
-      // the starts of later warps' ranges), waits for their count, and folds
-      // their partials into its own state in the MMA fragment layout: a
-      // log-sum-exp combine, then the output.
-      const int cf = wk, cl = cta_of(b - 1, T, W);
-      int others = 0;
-      for (int c = cf + 1; c <= cl; ++c) others += range_start(c, T, W) < range_start(c + 1, T, W);
-      unsigned int* cnt = p.ws.cnt + (int64_t)s * hkv + h;
-      bool ready = true;
-      if (lane == 0) {
-        const uint64_t t_start = dev::globaltimer_ns();
-        while (load_acquire(cnt) < (unsigned)others) {
-          if (dev::globaltimer_ns() - t_start > 2000000000ull) {  // bounded: flag and give up
-            atomicCAS(p.ws.err, 0, 1);
-            ready = false;
-            break;
-          }
-        }
-      }
-      ready = __shfl_sync(0xffffffffu, ready, 0);
-      __syncwarp();
-      // fold each contributor into this warp's state with a running
-      // log-sum-exp: its (max, sum) and its outputs are loaded together, so
-      // a contributor costs one round trip to L2
+      // the sequence's first piece: this warp finishes the (sequence, kv
+      // head).  If the context was cut by the end of this warp's range, the
+      // other pieces sit at the starts of later warps' ranges and finish
+      // first: wait for their count and fold their partials into this
+      // warp's state in the MMA fragment layout (a log-sum-exp combine).  A
+      // shared prefix's chunk partials (pa_decode_prefix) are folded the
+      // same way.  Then the output.
       float M0 = m0, M1 = m1, L0 = l0, L1 = l1;
-      for (int c = cf + 1; c <= cl && ready; ++c) {
-        if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
-        const float* pml = p.ws.ml + (int64_t)c * G * 2;
-        const float* po = p.ws.o + (int64_t)c * G * D;
+      // fold one partial: (max, sum) pairs and O rows of the group's query
+      // heads, column c at pml + 2c and po + c * D; its (max, sum) and its
+      // outputs are loaded together, so a partial costs one round trip to L2
+      auto fold = [&](const float* pml, const float* po) {
         const float mc0 = c0 < G ? __ldcg(pml + c0 * 2) : -INFINITY;
         const float mc1 = c1 < G ? __ldcg(pml + c1 * 2) : -INFINITY;
         const float lc0 = c0 < G ? __ldcg(pml + c0 * 2 + 1) : 0.f;
@@ -629,11 +701,44 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
         }
         M0 = n0;
         M1 = n1;
+      };
+      unsigned int* cnt = p.ws.cnt + (int64_t)s * hkv + h;
+      bool ready = true;
+      if (pe != b) {
+        const int cf = wk, cl = cta_of(b - 1, T, W);
+        int others = 0;
+        for (int c = cf + 1; c <= cl; ++c) others += range_start(c, T, W) < range_start(c + 1, T, W);
+        if (lane == 0) {
+          const uint64_t t_start = dev::globaltimer_ns();
+          const uint64_t limit = inject ? 1000000ull : 2000000000ull;
+          while (load_acquire(cnt) < (unsigned)others) {
+            if (dev::globaltimer_ns() - t_start > limit) {  // bounded: flag and give up
+              atomicCAS(p.ws.err, 0, 1);
+              ready = false;
+              break;
+            }
+          }
+        }
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        __syncwarp();
+        for (int c = cf + 1; c <= cl && ready; ++c) {
+          if (range_start(c, T, W) >= range_start(c + 1, T, W)) continue;
+          fold(p.ws.ml + (int64_t)c * G * 2, p.ws.o + (int64_t)c * G * D);
+        }
       }
-      // L0/L1 are whole-column sums already: l0/l1 were reduced over the
-      // warp above and a partial's sum is per column
+      if (skip > 0) {
+        // the shared prefix's chunks, computed for member slot j
+        const int j = __ldg(p.pfx_slot + s);
+        const int nch = (__ldg(p.pfx_blocks + __ldg(p.pfx_of + s)) + p.pfx_chunk_blocks - 1) / p.pfx_chunk_blocks;
+        for (int c = 0; c < nch; ++c) {
+          const int64_t prow = ((int64_t)c * p.pfx_members + j) * hq + (int64_t)h * G;
+          fold(p.pfx_ml + prow * 2, p.pfx_o + prow * D);
+        }
+      }
+      // L0/L1 are whole-column sums: l0/l1 were reduced over the warp above
+      // and a partial's sum is per column
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + obase;
-      const float i0 = p.out_scale / L0, i1 = p.out_scale / L1;
+      const float i0 = osc / L0, i1 = osc / L1;
 #pragma unroll
       for (int mt = 0; mt < C::DM; ++mt) {
         const int d0 = 16 * mt + g;
@@ -646,9 +751,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
           out[c1 * D + d0 + 8] = __float2bfloat16_rn(o[mt][3] * i1);
         }
       }
-      // ready for the next call (or a replay of this one)
-      __syncwarp();
-      if (lane == 0 && ready) *cnt = 0u;
+      if (pe != b) {
+        // ready for the next call (or a replay of this one)
+        __syncwarp();
+        if (lane == 0 && ready) *cnt = 0u;
+      }
     }
     t = pe;
   }
@@ -658,11 +765,18 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
   }
 }
 
+// Forward progress: a merging warp waits for pieces held by later CTAs, so
+// every CTA of the grid must be resident at once.  The grid is therefore
+// capped at the CTAs per SM that the runtime reports for this instance's
+// shared memory and registers, times the SMs.  (Two decode grids must not
+// run at the same time on one GPU: each could hold the SMs the other's later
+// CTAs wait for; the bounded wait would then end both with error word 1.)
 template <int KV, int D, int BS>
-cudaError_t launch_instance(const DecodeParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+cudaError_t launch_instance(DecodeParams p, const CUtensorMap& tm_k, const CUtensorMap& tm_v, int num_sms,
                             cudaStream_t stream) {
   using C = Cfg<KV, D, BS>;
-  const SmemLayout L = smem_layout(C::KVB + q_area_bytes(p.group, D), p.nstages, p.rows.num_seqs);
+  const SmemLayout L =
+      smem_layout(C::KVB + q_area_bytes(p.group, D), p.nstages, p.rows.num_seqs, p.pfx_of != nullptr);
   auto kern = decode_tc_kernel<KV, D, BS>;
   // raise the kernel's dynamic shared memory limit once per device
   static int set_for[64] = {0};
@@ -674,6 +788,20 @@ cudaError_t launch_instance(const DecodeParams& p, const CUtensorMap& tm_k, cons
     if (e != cudaSuccess) return e;
     if (dev < 64) set_for[dev] = (int)L.total;
   }
+  // resident CTAs per SM for this shared-memory size, queried once per
+  // device and size (host arithmetic only: allowed while a stream captures)
+  static int occ_smem[64] = {0}, occ_ctas[64] = {0};
+  int resident = dev < 64 && occ_smem[dev] == (int)L.total ? occ_ctas[dev] : 0;
+  if (resident == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kThreads, L.total);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) {
+      occ_smem[dev] = (int)L.total;
+      occ_ctas[dev] = resident;
+    }
+  }
+  if (resident < 1) return cudaErrorNotSupported;
+  if (p.grid > resident * num_sms) p.grid = resident * num_sms;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -691,19 +819,19 @@ cudaError_t launch_instance(const DecodeParams& p, const CUtensorMap& tm_k, cons
 
 int decode_tc_workers(int num_sms) { return kMaxCtasPerSM * num_sms * kWarps; }
 
-size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages) {
+size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages, bool pfx) {
   const int elem = kv == kFP8 ? 1 : 2;
   const int stage = 2 * block_size * head_dim * elem + q_area_bytes(group, head_dim);
-  return smem_layout(stage, nstages, num_seqs).total;
+  return smem_layout(stage, nstages, num_seqs, pfx).total;
 }
 
 // Ring stages per warp that fit `ctas` CTAs per SM.
-static int pick_stages(int kv, int head_dim, int block_size, int group, int num_seqs, int ctas) {
+static int pick_stages(int kv, int head_dim, int block_size, int group, int num_seqs, bool pfx, int ctas) {
   const int elem = kv == kFP8 ? 1 : 2;
   const int stage = 2 * block_size * head_dim * elem + q_area_bytes(group, head_dim);
   // 1 KB per CTA is reserved, plus a little static shared memory
   const int budget = kSmemPerSM / ctas - 1024 - 64;
-  const int fixed = (int)smem_layout(stage, 0, num_seqs).total;
+  const int fixed = (int)smem_layout(stage, 0, num_seqs, pfx).total;
   int n = (budget - fixed) / (kWarps * (stage + 8 + 16));
   if (n > kMaxStagesPerWarp) n = kMaxStagesPerWarp;
   return n;
@@ -725,19 +853,19 @@ cudaError_t launch_decode_tc(const DecodeParams& p_in, const CUtensorMap& tm_k, 
   // ring, else fewer CTAs with deeper rings (large blocks)
   int ctas = kv == kFP8 ? ctas_per_sm<kFP8>() : ctas_per_sm<kBF16>();
   for (;; --ctas) {
-    p.nstages = pick_stages(kv, head_dim, block_size, p.group, p.rows.num_seqs, ctas);
+    p.nstages = pick_stages(kv, head_dim, block_size, p.group, p.rows.num_seqs, p.pfx_of != nullptr, ctas);
     if (p.nstages >= 2 || ctas == 1) break;
   }
   if (p.nstages < 2) return cudaErrorNotSupported;
   p.grid = ctas * num_sms;
   if (kv == kBF16) {
-    if (head_dim == 128 && block_size == 16) return launch_instance<kBF16, 128, 16>(p, tm_k, tm_v, stream);
-    if (head_dim == 128 && block_size == 32) return launch_instance<kBF16, 128, 32>(p, tm_k, tm_v, stream);
-    if (head_dim == 64 && block_size == 16) return launch_instance<kBF16, 64, 16>(p, tm_k, tm_v, stream);
-    if (head_dim == 64 && block_size == 32) return launch_instance<kBF16, 64, 32>(p, tm_k, tm_v, stream);
+    if (head_dim == 128 && block_size == 16) return launch_instance<kBF16, 128, 16>(p, tm_k, tm_v, num_sms, stream);
+    if (head_dim == 128 && block_size == 32) return launch_instance<kBF16, 128, 32>(p, tm_k, tm_v, num_sms, stream);
+    if (head_dim == 64 && block_size == 16) return launch_instance<kBF16, 64, 16>(p, tm_k, tm_v, num_sms, stream);
+    if (head_dim == 64 && block_size == 32) return launch_instance<kBF16, 64, 32>(p, tm_k, tm_v, num_sms, stream);
   } else if (kv == kFP8) {
-    if (head_dim == 128 && block_size == 16) return launch_instance<kFP8, 128, 16>(p, tm_k, tm_v, stream);
-    if (head_dim == 128 && block_size == 32) return launch_instance<kFP8, 128, 32>(p, tm_k, tm_v, stream);
+    if (head_dim == 128 && block_size == 16) return launch_instance<kFP8, 128, 16>(p, tm_k, tm_v, num_sms, stream);
+    if (head_dim == 128 && block_size == 32) return launch_instance<kFP8, 128, 32>(p, tm_k, tm_v, num_sms, stream);
   }
   return cudaErrorNotSupported;
 }

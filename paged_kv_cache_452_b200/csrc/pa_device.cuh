@@ -1,6 +1,6 @@
 // Device-side building blocks for the sm_100a kernels: mbarriers, TMA and
 // bulk copies, warp-level matrix loads/moves, tensor-core MMA, conversions.
-// Everything here is a thin wrapper over one documented PTX instruction.
+// Everything here is a thin wrapper over one or two documented PTX instructions.
 #pragma once
 
 #include <cuda.h>
@@ -231,18 +231,29 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
   return __uint_as_float(bits16 << 16);
 }
 
-// Four e4m3 bytes -> two f16x2 words holding the same values times 2^-8,
-// exactly (normals and subnormals alike; the e4m3 NaN code is not handled).
-// An e4m3 byte s.eeee.mmm placed at f16 bits 15 and 13..7 reads as
-// 2^(eeee-15) * 1.mmm (or 0.mmm * 2^-14 when eeee = 0): the e4m3 value
-// scaled by 2^-8, because the exponent biases differ by 8.  Adding the sign
-// bit to itself before the shift carries it past the zero bit 14.
-// lo = bytes (0, 2), hi = bytes (1, 3) of w.
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t x0 = w & 0x00FF00FFu;
-  const uint32_t x1 = (w >> 8) & 0x00FF00FFu;
-  lo = (x0 + (x0 & 0x00800080u)) << 7;
-  hi = (x1 + (x1 & 0x00800080u)) << 7;
+// Four e4m3 bytes -> two f16x2 words with the same values (f16 holds every
+// e4m3 value exactly; NaN codes become NaN), by the hardware's paired
+// conversion: lo = (byte 0, byte 1), hi = (byte 2, byte 3) of w, lower byte
+// in the lower half.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+// Two fp32 values -> two e4m3 codes (round to nearest even, saturating to
+// +-448; NaN stays NaN): lo in the lower byte.  cvt packs its first source
+// operand into the upper byte.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// One e4m3 byte -> its value as fp32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}" : "=r"(h2) : "r"(byte & 0xFFu));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
 }  // namespace dev

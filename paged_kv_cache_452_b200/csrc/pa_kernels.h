@@ -19,6 +19,8 @@ struct CacheWriteParams {
   int32_t num_tokens, num_kv_heads, head_dim, block_size;
   int64_t num_slots;  // num_blocks * block_size
   float k_scale, v_scale;
+  const float* k_head;  // per-kv-head scales (device) or nullptr: k_scale / v_scale
+  const float* v_head;
 };
 cudaError_t launch_cache_write(const CacheWriteParams& p, int in_dtype, int kv_dtype, cudaStream_t stream);
 
@@ -65,15 +67,34 @@ struct DecodeParams {
   int32_t num_blocks;  // table entries outside [0, num_blocks) are flagged and read as block 0
   int32_t nstages;
   int32_t grid;
-  float scale_log2;  // softmax scale * log2(e), times the K dequant factor for fp8
-  float out_scale;   // 1, or the V dequant factor for fp8
+  float scale_log2;  // softmax scale * log2(e), times the per-tensor K dequant factor for fp8
+  float out_scale;   // 1, or the per-tensor V dequant factor for fp8
+  const float* k_head;  // fp8 per-kv-head scales (device; they multiply scale_log2 / out_scale) or nullptr
+  const float* v_head;
+  // fused cache write (pa_decode_fused): the new token's rows [rows][Hkv][D]
+  // (bf16) and the pools to store them in; k_new == nullptr: no write
+  const uint8_t* k_new;
+  const uint8_t* v_new;
+  uint8_t* k_pool;
+  uint8_t* v_pool;
+  float k_scale_w, v_scale_w;  // per-tensor quantisation scales of the write (fp8)
+  // shared prefixes (pa_decode_prefix; pfx_of == nullptr: none): sequence s
+  // with pfx_of[s] = p >= 0 skips the first pfx_blocks[p] blocks of its row
+  // and folds the chunk partials of member slot pfx_slot[s] into its result
+  const int32_t* pfx_of;
+  const int32_t* pfx_slot;
+  const int32_t* pfx_blocks;
+  const float* pfx_ml;  // [chunks][num_members][Hq][2]
+  const float* pfx_o;   // [chunks][num_members][Hq][D]
+  int32_t pfx_members;
+  int32_t pfx_chunk_blocks;  // blocks per chunk (kPrefixChunkKeys / block_size)
   DecodeWorkspace ws;
 };
 
 // kv: kBF16 or kFP8; returns cudaErrorNotSupported for unsupported shapes.
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                              int kv, int head_dim, int block_size, int num_sms, cudaStream_t stream);
-size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages);
+size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages, bool pfx);
 int decode_tc_workers(int num_sms);  // the most worker warps a launch can have (workspace sizing)
 size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms);
 
@@ -89,7 +110,23 @@ struct PrefillParams {
   int32_t nstages_v;  // the tcgen05 kernel's V stages
   float scale_log2;
   int32_t* err;  // workspace error word
+  // Shared-prefix mode of the tcgen05 kernel (pa_decode_prefix): units are
+  // (prefix, kv head, tile of members, chunk of prefix keys) and each writes
+  // partial (max reference, sum, unnormalised O) rows instead of outputs.
+  // rows.num_seqs then counts prefixes; the other rows fields are unused.
+  const int32_t* pfx_start;    // [P + 1] CSR into pfx_members
+  const int32_t* pfx_members;  // [M] sequence of each member slot (= its decode row)
+  const int32_t* pfx_blocks;   // [P] blocks in each prefix
+  int32_t num_members;         // M
+  int32_t chunk_keys;          // prefix keys per unit, a multiple of 128
+  float* pfx_ml;               // [chunks][M][Hq][2] (max reference, sum), log2 domain
+  float* pfx_o;                // [chunks][M][Hq][D]
 };
+
+// The split of a prefix into chunks of keys that pa_decode_prefix uses.
+constexpr int kPrefixChunkKeys = 256;
+cudaError_t launch_prefix_umma(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                               int head_dim, int block_size, int num_sms, cudaStream_t stream);
 bool prefill_tc_supported(int kv, int q, int head_dim, int block_size, int group);
 // The same rows on tcgen05 (TMEM accumulators); cudaErrorNotSupported when
 // the shape or the batch's unit table does not fit (the caller falls back).
@@ -110,6 +147,8 @@ struct SimtParams {
   int32_t num_q_heads, num_kv_heads, head_dim, block_size;
   float scale;
   float k_scale, v_scale;
+  const float* k_head;  // fp8 per-kv-head scales (device) or nullptr: k_scale / v_scale
+  const float* v_head;
   int32_t only_multi_row;  // 1: skip sequences with exactly one query row
   int32_t num_blocks;      // table entries outside [0, num_blocks) are flagged and read as block 0
   int32_t* err;            // error word of the caller's workspace

@@ -354,4 +354,69 @@ int pa_pool_free_order(const pa_pool* pool, int32_t* out, int32_t cap, int32_t* 
   return PA_OK;
 }
 
+int pa_prefix_groups(const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                     int32_t num_seqs, int32_t block_size, int32_t* prefix_start, int32_t* prefix_members,
+                     int32_t* prefix_blocks, int32_t* seq_prefix, int32_t* seq_slot, int32_t* num_prefixes,
+                     int32_t* num_members) {
+  pa::clear_error();
+  if (num_seqs < 0 || max_blocks_per_seq < 0 || block_size <= 0)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_prefix_groups: bad sizes");
+  if (!num_prefixes || !num_members || (num_seqs > 0 && (!block_tables || !seq_lens || !prefix_start ||
+                                                         !prefix_members || !prefix_blocks || !seq_prefix ||
+                                                         !seq_slot)))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_prefix_groups: NULL pointer");
+  // blocks sequence s could share: whole blocks before the one holding its
+  // last token, within its table row
+  auto cap = [&](int s) {
+    const int32_t len = seq_lens[s];
+    if (len <= 0) return 0;
+    const int32_t c = (len - 1) / block_size;
+    return c < max_blocks_per_seq ? c : max_blocks_per_seq;
+  };
+  const int32_t* row0 = block_tables;
+  auto row = [&](int s) { return row0 + (int64_t)s * max_blocks_per_seq; };
+  // candidates grouped by their first physical block, in order of first appearance
+  std::unordered_map<int32_t, int32_t> group_of_block;
+  std::vector<std::vector<int32_t>> groups;
+  for (int s = 0; s < num_seqs; ++s) {
+    seq_prefix[s] = -1;
+    seq_slot[s] = -1;
+    if (cap(s) < 1) continue;
+    auto it = group_of_block.find(row(s)[0]);
+    if (it == group_of_block.end()) {
+      group_of_block.emplace(row(s)[0], (int32_t)groups.size());
+      groups.push_back({s});
+    } else {
+      groups[it->second].push_back(s);
+    }
+  }
+  int32_t np = 0, nm = 0;
+  prefix_start[0] = 0;
+  for (const auto& g : groups) {
+    if (g.size() < 2) continue;
+    // the longest leading run of blocks every member has in common
+    int32_t common = cap(g[0]);
+    for (size_t k = 1; k < g.size(); ++k) {
+      const int32_t c = cap(g[k]);
+      if (c < common) common = c;
+      int32_t i = 0;
+      while (i < common && row(g[k])[i] == row(g[0])[i]) ++i;
+      common = i;
+    }
+    if (common < 1) continue;
+    prefix_blocks[np] = common;
+    for (size_t k = 0; k < g.size(); ++k) {
+      prefix_members[nm] = g[k];
+      seq_prefix[g[k]] = np;
+      seq_slot[g[k]] = nm;
+      ++nm;
+    }
+    ++np;
+    prefix_start[np] = nm;
+  }
+  *num_prefixes = np;
+  *num_members = nm;
+  return PA_OK;
+}
+
 }  // extern "C"

@@ -109,7 +109,11 @@ __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int ns
 // Byte offset of 16-byte unit u of row r in a 128-byte-swizzled chunk.
 __device__ __forceinline__ uint32_t swz(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-template <int D, int BS>
+// PFX: the shared-prefix mode (pa_decode_prefix): a unit is (prefix, kv
+// head, 128 / G member sequences, one chunk of the prefix's keys); its rows
+// are the members' decode queries, every prefix key is visible to every row,
+// and it writes partial (max reference, sum, unnormalised O) rows.
+template <int D, int BS, bool PFX>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_umma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const PrefillParams p) {
@@ -134,10 +138,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int QB = kRows / G;  // query positions per unit
 
   dev::grid_dep_wait();
-  // ---- query blocks per prompt sequence, exclusive prefix ---------------------
+  // ---- units per prompt sequence (per prefix), exclusive prefix ---------------
   for (int s = tid; s < S; s += kThreads) {
-    const int qlen = p.rows.qsl[s + 1] - p.rows.qsl[s];
-    prefix[s] = qlen > 1 ? (qlen + QB - 1) / QB : 0;
+    if constexpr (PFX) {
+      const int nm = p.pfx_start[s + 1] - p.pfx_start[s];
+      const int nc = (p.pfx_blocks[s] * BS + p.chunk_keys - 1) / p.chunk_keys;
+      prefix[s] = ((nm + QB - 1) / QB) * nc;
+    } else {
+      const int qlen = p.rows.qsl[s + 1] - p.rows.qsl[s];
+      prefix[s] = qlen > 1 ? (qlen + QB - 1) / QB : 0;
+    }
   }
   __syncthreads();
   {
@@ -170,8 +180,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Units are processed persistently: this CTA takes ordinals blockIdx.x,
   // blockIdx.x + gridDim.x, ...  Ordinal i is query block i / Hkv (a
   // sequence's last query blocks first) of kv head i % Hkv.
+  // A unit's rows are query rows first + q0 .. first + q0 + qn - 1 (in PFX
+  // mode: member slots first .. first + qn - 1); its keys are blocks
+  // blk0 .. blk0 + nbneed - 1 of sequence s's table row.
   struct Unit {
-    int s, h, first, q0, qn, pos0, seq_len, nbneed, ntiles;
+    int s, h, first, q0, qn, pos0, seq_len, nbneed, ntiles, blk0, chunk;
   };
   auto unit_of = [&](int idx) {
     Unit u;
@@ -181,8 +194,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mid = (lo + hi + 1) >> 1;
       if (prefix[mid] <= ub) lo = mid; else hi = mid - 1;
     }
-    u.s = lo;
     u.h = idx % hkv;
+    if constexpr (PFX) {
+      // prefix lo: member tile mt, key chunk c
+      const int nkeys = p.pfx_blocks[lo] * BS;
+      const int nc = (nkeys + p.chunk_keys - 1) / p.chunk_keys;
+      const int local = ub - prefix[lo];
+      const int mt = local / nc;
+      u.chunk = local - mt * nc;
+      const int m0 = p.pfx_start[lo], nm = p.pfx_start[lo + 1] - m0;
+      u.s = p.pfx_members[m0];  // every member's row holds the prefix's blocks
+      u.first = m0 + mt * QB;
+      u.q0 = 0;
+      u.qn = min(QB, nm - mt * QB);
+      u.pos0 = 1 << 30;  // no causal limit: every prefix key is visible
+      const int kbeg = u.chunk * p.chunk_keys;
+      u.seq_len = min(p.chunk_keys, nkeys - kbeg);  // keys of this chunk
+      u.blk0 = kbeg / BS;
+      u.nbneed = u.seq_len / BS;
+      if (u.blk0 + u.nbneed > p.max_blocks) {
+        if (warp == 2 && lane == 0) atomicCAS(p.err, 0, 3);
+        u.nbneed = max(0, p.max_blocks - u.blk0);
+      }
+      u.ntiles = (u.seq_len + kKeys - 1) / kKeys;
+      return u;
+    }
+    u.s = lo;
+    u.blk0 = 0;
+    u.chunk = 0;
     const int qb = prefix[lo + 1] - prefix[lo] - 1 - (ub - prefix[lo]);
     u.first = p.rows.qsl[lo];
     const int qlen = p.rows.qsl[lo + 1] - u.first;
@@ -242,7 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a tile
     auto entry = [&](const Unit& u, int k) -> int32_t {
       const int b = k * C::BPT + j;
-      return (lane < C::BOXES && b < u.nbneed) ? __ldg(p.block_tables + (int64_t)u.s * p.max_blocks + b) : -2;
+      return (lane < C::BOXES && b < u.nbneed) ? __ldg(p.block_tables + (int64_t)u.s * p.max_blocks + u.blk0 + b)
+                                                : -2;
     };
     bool ok = true;
     int g = 0;
@@ -357,7 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit u = unit_of(idx);
       const bool valid = r < u.qn * G;
       const int pos = u.pos0 + u.q0 + r / G;  // the row's position: keys <= pos
-      const int64_t grow = ((int64_t)(u.first + u.q0 + r / G) * hq + (int64_t)u.h * G + r % G) * D;
+      // the row's query: row first + q0 + r / G, or (PFX) the decode row of
+      // member slot first + r / G
+      const int qrow = !PFX ? u.first + u.q0 + r / G : (valid ? __ldg(p.pfx_members + u.first + r / G) : 0);
+      const int64_t grow = ((int64_t)qrow * hq + (int64_t)u.h * G + r % G) * D;
       // ---- this half of the Q row into the swizzled Q tile (zero for rows
       // past the unit); the previous unit's MMAs have all completed (its
       // output was read after them)
@@ -474,6 +517,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         xsum[hh * 128 + r] = lsum;
         dev::named_bar_sync(pair_bar, 64);
         const float total = lsum + xsum[(hh ^ 1) * 128 + r];
+        if constexpr (PFX) {
+          // partial row of member slot first + r / G, q head h * G + r % G:
+          // (max reference, sum) and this half of the unnormalised O
+          const int64_t prow =
+              ((int64_t)u.chunk * p.num_members + u.first + r / G) * hq + (int64_t)u.h * G + r % G;
+          if (valid && ok && hh == 0) *reinterpret_cast<float2*>(p.pfx_ml + prow * 2) = make_float2(ref, total);
+          float4* dst = reinterpret_cast<float4*>(p.pfx_o + prow * D + HD * hh);
+#pragma unroll 1
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t w[32];
+            dev::tmem_ld32(t_o + (uint32_t)(HD * hh + 32 * c) + lane_addr, w);
+            if (valid && ok) {
+#pragma unroll
+              for (int uu = 0; uu < 8; ++uu)
+                dst[8 * c + uu] = make_float4(__uint_as_float(w[4 * uu]), __uint_as_float(w[4 * uu + 1]),
+                                              __uint_as_float(w[4 * uu + 2]), __uint_as_float(w[4 * uu + 3]));
+            }
+          }
+        } else {
         const float inv = valid ? 1.f / total : 0.f;
         uint4* dst = reinterpret_cast<uint4*>(p.out + (grow + HD * hh) * 2);
 #pragma unroll 1
@@ -492,6 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        }
       }
       dev::tc_fence_before();
       __syncwarp();
@@ -509,12 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int BS>
+template <int D, int BS, bool PFX = false>
 cudaError_t launch_u(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v, int grid,
                      cudaStream_t stream) {
   using C = U<D, BS>;
   const ULayout L = u_layout(C::QBYTES, C::KVT, p.nstages, p.nstages_v, p.rows.num_seqs);
-  auto kern = prefill_umma_kernel<D, BS>;
+  auto kern = prefill_umma_kernel<D, BS, PFX>;
   static int set_for[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -563,6 +626,31 @@ cudaError_t launch_prefill_umma(const PrefillParams& p_in, const CUtensorMap& tm
   if (head_dim == 128 && block_size == 32) return launch_u<128, 32>(p, tm_k, tm_v, (int)grid, stream);
   if (head_dim == 64 && block_size == 16) return launch_u<64, 16>(p, tm_k, tm_v, (int)grid, stream);
   if (head_dim == 64 && block_size == 32) return launch_u<64, 32>(p, tm_k, tm_v, (int)grid, stream);
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_prefix_umma(const PrefillParams& p_in, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                               int head_dim, int block_size, int num_sms, cudaStream_t stream) {
+  PrefillParams p = p_in;
+  const int nch = head_dim / 64;
+  const int qbytes = nch * kChunk, kvt = nch * kChunk;
+  const int fixed = (int)u_layout(qbytes, kvt, 0, 0, p.rows.num_seqs).total;
+  const int nbuf = (kSmemOptIn - fixed) / (kvt + 16);
+  const int nsk = min(4, nbuf / 2), nsv = min(4, nbuf - nbuf / 2);
+  if (nsk < 2 || nsv < 2) return cudaErrorNotSupported;
+  p.nstages = nsk;
+  p.nstages_v = nsv;
+  // units: at most (member tiles) x (chunks) x kv heads; the exact count is
+  // the kernel's, CTAs past it return at once
+  const int qb = kRows / p.group;
+  const int64_t chunks = ((int64_t)p.max_blocks * block_size + p.chunk_keys - 1) / p.chunk_keys;
+  const int64_t bound = ((int64_t)p.num_members / qb + p.rows.num_seqs) * chunks * p.num_kv_heads;
+  if (bound <= 0) return cudaSuccess;
+  const int64_t grid = bound < num_sms ? bound : num_sms;
+  if (head_dim == 128 && block_size == 16) return launch_u<128, 16, true>(p, tm_k, tm_v, (int)grid, stream);
+  if (head_dim == 128 && block_size == 32) return launch_u<128, 32, true>(p, tm_k, tm_v, (int)grid, stream);
+  if (head_dim == 64 && block_size == 16) return launch_u<64, 16, true>(p, tm_k, tm_v, (int)grid, stream);
+  if (head_dim == 64 && block_size == 32) return launch_u<64, 32, true>(p, tm_k, tm_v, (int)grid, stream);
   return cudaErrorNotSupported;
 }
 

@@ -12,9 +12,9 @@ from typing import List, Optional
 import numpy as np
 import torch
 
-from . import (PA_FP8_E4M3, BlockPool, CacheDesc, alloc_cache, alloc_workspace, default_scale,
-               pa_cache_write, pa_decode, pa_decode_chunked_prefill, pa_decode_workspace_size,
-               pa_prefill_workspace_size)
+from . import (PA_FP8_E4M3, BlockPool, CacheDesc, PrefixGroups, alloc_cache, alloc_workspace, default_scale,
+               pa_cache_write, pa_decode, pa_decode_chunked_prefill, pa_decode_fused, pa_decode_prefix,
+               pa_decode_prefix_workspace_size, pa_decode_workspace_size, pa_prefill_workspace_size)
 
 # sentinel stored in unwritten cache elements so a stray read shows up
 _SENTINEL = {0: float("nan"), 1: float("nan"), 2: 0x7F}
@@ -47,9 +47,17 @@ class DeviceBatch:
         return self.qsl is None
 
 
-def _desc_for(wl):
+def _desc_for(wl, device=None):
+    """The pool's desc; per-kv-head e4m3 scales (an array in the workload)
+    go to the device as fp32 tensors that the desc keeps alive."""
+    ks, vs = wl.k_scale, wl.v_scale
+    kh = vh = None
+    if np.ndim(ks) == 1:
+        kh, ks = torch.from_numpy(np.asarray(ks, dtype=np.float32)).to(device), 1.0
+    if np.ndim(vs) == 1:
+        vh, vs = torch.from_numpy(np.asarray(vs, dtype=np.float32)).to(device), 1.0
     return CacheDesc.make(wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.num_q_heads, wl.head_dim,
-                          wl.kv_dtype, wl.q_dtype, wl.k_scale, wl.v_scale)
+                          wl.kv_dtype, wl.q_dtype, ks, vs, kh, vh)
 
 
 def setup(wl, device, write_chunk_tokens: int = 1 << 18) -> DeviceBatch:
@@ -71,7 +79,7 @@ def setup(wl, device, write_chunk_tokens: int = 1 << 18) -> DeviceBatch:
     # e4m3 pool needs its per-tensor scales (the drawn values' amax) before
     # anything is quantised, so its context is staged on the device and
     # written once every draw is in.
-    desc = _desc_for(wl)
+    desc = _desc_for(wl, device)
     k_cache, v_cache = alloc_cache(desc, device, fill=_SENTINEL[desc.kv_dtype])
     staged, staged_tokens = [], 0
     for s, (k, v) in enumerate(_draws_in_order(wl, S)):
@@ -84,7 +92,7 @@ def setup(wl, device, write_chunk_tokens: int = 1 << 18) -> DeviceBatch:
             staged, staged_tokens = [], 0
     if fp8:
         wl.fp8_scales_from_draws()
-        desc = _desc_for(wl)
+        desc = _desc_for(wl, device)
     _write_staged(desc, staged, k_cache, v_cache)
 
     max_blocks = max(1, max(-(-(int(wl.context_lens[s]) + int(wl.q_lens[s])) // wl.block_size)
@@ -111,6 +119,19 @@ def setup(wl, device, write_chunk_tokens: int = 1 << 18) -> DeviceBatch:
         prior_slots=prior_slots, num_cached=num_cached)
     torch.cuda.synchronize(device)
     return batch
+
+
+def clone(b: DeviceBatch) -> DeviceBatch:
+    """A second copy of a batch on the same device: its own K/V pools (device
+    copies of b's), output and zeroed workspace; the step inputs and the host
+    pool are shared.  Cheaper than drawing the workload again."""
+    import copy
+    c = copy.copy(b)
+    c.k_cache = b.k_cache.clone()
+    c.v_cache = b.v_cache.clone()
+    c.out = torch.empty_like(b.out)
+    c.workspace = torch.zeros_like(b.workspace)
+    return c
 
 
 def _draws_in_order(wl, S, window=None):
@@ -153,3 +174,37 @@ def attend(b: DeviceBatch, stream=None):
 def step(b: DeviceBatch, stream=None):
     write_step(b, stream)
     attend(b, stream)
+
+
+@dataclass
+class PrefixPlan:
+    groups: PrefixGroups
+    dev: dict
+    workspace: torch.Tensor
+
+
+def prefix_plan(b: DeviceBatch) -> PrefixPlan:
+    """The batch's shared prefixes (from its block tables) and the workspace
+    pa_decode_prefix needs, on b's device."""
+    dev = b.tables.device
+    groups = PrefixGroups(b.tables_host, b.seq_lens, b.desc.block_size)
+    ws = pa_decode_prefix_workspace_size(b.desc, b.seq_lens.shape[0], groups.num_members, groups.max_prefix_blocks)
+    return PrefixPlan(groups, groups.to(dev), alloc_workspace(ws, dev))
+
+
+def attend_prefix(b: DeviceBatch, plan: PrefixPlan, stream=None):
+    """pa_decode_prefix: each shared prefix attended once for its sequences."""
+    pa_decode_prefix(b.desc, b.q, b.k_cache, b.v_cache, b.tables, b.seq_lens, plan.groups, plan.dev, b.scale, b.out,
+                     plan.workspace, stream)
+
+
+def step_prefix(b: DeviceBatch, plan: PrefixPlan, stream=None):
+    write_step(b, stream)
+    attend_prefix(b, plan, stream)
+
+
+def step_fused(b: DeviceBatch, stream=None):
+    """The same step as one launch: pa_decode_fused writes each sequence's
+    new token and attends (pure decode steps on the tensor-core path)."""
+    pa_decode_fused(b.desc, b.q, b.k_new, b.v_new, b.k_cache, b.v_cache, b.tables, b.seq_lens, b.scale, b.out,
+                    b.workspace, stream)

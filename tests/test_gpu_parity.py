@@ -125,6 +125,22 @@ EDGE = {
     # groups whose (max, sum) block is not a multiple of 16 bytes
     "split_group3": dict(context_lens=[5000] * 8 + [3, 40], num_q_heads=6, num_kv_heads=2),
     "split_group7_head64": dict(context_lens=[5000] * 8 + [0, 16], num_q_heads=14, num_kv_heads=2, head_dim=64),
+    # e4m3 pools with one scale per kv head: heads about 3 000x apart, so a
+    # head that used another head's scale would saturate or vanish; some
+    # small scales saturate the codes at +-448 (the oracle does the same)
+    "fp8_head_scales": dict(context_lens=[0, 5, 80, 300, 17], kv_dtype="e4m3", num_q_heads=16, num_kv_heads=4,
+                            scale_mode="fixed", k_scale=[0.001, 0.01, 3.0, 0.5], v_scale=[2.0, 0.0007, 0.05, 1.0]),
+    "fp8_head_scales_split": dict(context_lens=[3000] * 15 + [17], kv_dtype="e4m3", num_q_heads=32, num_kv_heads=8,
+                                  scale_mode="fixed", k_scale=[0.001, 0.3, 3.0, 0.02, 0.01, 1.0, 0.1, 0.005],
+                                  v_scale=[0.05, 2.0, 0.0007, 0.01, 0.3, 0.02, 1.5, 0.1]),
+    "fp8_head_scales_from_draws_bs32": dict(context_lens=[31, 32, 33, 200], kv_dtype="e4m3", block_size=32,
+                                            scale_mode="head"),
+    # per-head scales on the CUDA-core path: fp32 queries, and a group above 8
+    "fp8_head_scales_f32_queries": dict(context_lens=[9, 70], kv_dtype="e4m3", q_dtype="f32", num_q_heads=4,
+                                        num_kv_heads=2, scale_mode="fixed", k_scale=[0.002, 2.0],
+                                        v_scale=[3.0, 0.001]),
+    "fp8_head_scales_group16": dict(context_lens=[7, 100], kv_dtype="e4m3", num_q_heads=32, num_kv_heads=2,
+                                    scale_mode="fixed", k_scale=[0.002, 2.0], v_scale=[3.0, 0.001]),
 }
 
 
@@ -150,6 +166,8 @@ MIXED_EDGE = {
     "group3_prefill": dict(context_lens=[4, 0], q_lens=[9, 22], num_q_heads=6, num_kv_heads=2),  # CUDA cores
     "prefill_only": dict(context_lens=[0, 200], q_lens=[33, 100]),
     "fp8_prefill": dict(context_lens=[0, 40], q_lens=[17, 30], kv_dtype="e4m3"),  # CUDA cores
+    "fp8_head_scales_prefill": dict(context_lens=[0, 40, 9], q_lens=[17, 30, 1], kv_dtype="e4m3", num_q_heads=8,
+                                    num_kv_heads=2, scale_mode="fixed", k_scale=[0.01, 1.0], v_scale=[0.3, 0.003]),
     # more prompt units than SMs: persistent CTAs chain several units
     "many_units": dict(context_lens=[7 * i for i in range(40)] + [5, 9], q_lens=[40] * 40 + [1, 1],
                        num_q_heads=8, num_kv_heads=2),
@@ -266,3 +284,30 @@ def test_workload_full_size_sampled(name, seqs, cuda_device):
     """Full-size workload, launched exactly as bench.py does; the oracle checks
     sampled sequences (their rows, their cache bytes) and the full tables."""
     run_and_check(W.make(name, "full"), cuda_device, seqs)
+
+
+def test_merge_wait_that_runs_out_is_reported_and_the_next_call_is_correct(cuda_device):
+    """Failure detection without a GPU fault: the workspace's fault-injection
+    word makes the later pieces of every cut context skip their count-in,
+    so each merging warp's bounded wait runs out (after 1 ms) and sets error
+    word 1.  The call returns, the context stays usable, and once the
+    workspace is zeroed again the next call gives the same bits as before."""
+    import time
+    wl = W.custom("merge_timeout", context_lens=[2000] * 20, num_q_heads=32, num_kv_heads=8)
+    b = runner.setup(wl, cuda_device)
+    runner.step(b)
+    torch.cuda.synchronize()
+    assert pa.workspace_error(b.workspace) == 0
+    ref = b.out.clone()
+    b.workspace.view(torch.int32)[1] = 1
+    t0 = time.perf_counter()
+    runner.attend(b)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert pa.workspace_error(b.workspace) == 1
+    assert elapsed < 1.0, f"the injected wait should end after about 1 ms, took {elapsed:.3f} s"
+    b.workspace.zero_()
+    runner.attend(b)
+    torch.cuda.synchronize()
+    assert pa.workspace_error(b.workspace) == 0
+    assert torch.equal(b.out.view(torch.int16), ref.view(torch.int16))

@@ -109,3 +109,74 @@ def test_decode_rejects_bad_arguments_on_host():
     assert rc == 1 and b"misaligned" in L.pa_last_error()
     rc = L.pa_decode(ctypes.byref(desc), None, p, p, p, 4, p, 3, 1.0, p, p, 1 << 20, None)
     assert rc == 1
+
+
+def test_static_decode_checks_arguments_before_touching_its_scratch():
+    """pa_decode_static refuses what pa_decode refuses, on the host, before
+    it clears any scratch: a batch past 16384 sequences (whatever its
+    scratch size: a CUDA-core desc needs only the 256-byte error word),
+    NULL or misaligned pointers."""
+    L = pa.lib()
+    p = 256
+    simt = pa.CacheDesc.make(16, 16, 128, 128, 64, "f32", "f32")  # group 1: the CUDA-core path
+    rc = L.pa_decode_static(ctypes.byref(simt), p, p, p, p, 1, p, 16385, 1.0, p, None)
+    assert rc == 2 and b"16384" in L.pa_last_error()
+    tc = pa.CacheDesc.make(16, 16, 2, 8, 128, "bf16", "bf16")
+    assert L.pa_decode_static(ctypes.byref(tc), p, p, p, p, 1, p, 20000, 1.0, p, None) == 2
+    assert L.pa_decode_static(ctypes.byref(tc), None, p, p, p, 1, p, 3, 1.0, p, None) == 1
+    assert L.pa_decode_static(ctypes.byref(tc), p + 2, p, p, p, 1, p, 3, 1.0, p, None) == 1
+    assert b"misaligned" in L.pa_last_error()
+    assert L.pa_decode_static(ctypes.byref(tc), p, p, p, p, 1, p, 0, 1.0, p, None) == 0  # empty batch
+    assert L.pa_decode_static(None, p, p, p, p, 1, p, 3, 1.0, p, None) == 1
+
+
+def _groups_model(tables, lens, bs):
+    """Plain restatement of the grouping rule: sequences whose rows start
+    with the same block, two or more; the prefix is the longest leading run
+    every member shares, cut to keep each member's last token outside."""
+    cap = [0 if n <= 0 else min((n - 1) // bs, len(r)) for r, n in zip(tables, lens)]
+    by_first = {}
+    for s, r in enumerate(tables):
+        if cap[s] >= 1:
+            by_first.setdefault(r[0], []).append(s)
+    out = []
+    for mem in sorted(by_first.values(), key=lambda m: m[0]):
+        if len(mem) < 2:
+            continue
+        k = min(cap[s] for s in mem)
+        while k > 0 and any(tables[s][:k] != tables[mem[0]][:k] for s in mem):
+            k -= 1
+        if k >= 1:
+            out.append((mem, k))
+    return out
+
+
+def test_prefix_groups_match_a_plain_model():
+    import numpy as np
+    import torch
+    g = np.random.default_rng(7)
+    for trial in range(200):
+        bs = int(g.choice([16, 32]))
+        n = int(g.integers(0, 12))
+        width = 8
+        base = [list(g.permutation(100)[:width]) for _ in range(3)]
+        tables, lens = [], []
+        for _ in range(n):
+            r = list(base[int(g.integers(0, 3))]) if g.random() < 0.7 else list(g.permutation(100)[:width] + 100)
+            cut = int(g.integers(0, width + 1))
+            r[cut:] = list(g.permutation(100)[:width - cut] + 200)
+            tables.append(r)
+            lens.append(int(g.integers(0, width * bs + 1)))
+        bt = torch.tensor(tables, dtype=torch.int32).reshape(n, width)
+        grp = pa.PrefixGroups(bt, torch.tensor(lens, dtype=torch.int32), bs)
+        want = _groups_model([list(map(int, r)) for r in tables], lens, bs)
+        got = []
+        for p in range(grp.num_prefixes):
+            mem = grp.prefix_members[int(grp.prefix_start[p]):int(grp.prefix_start[p + 1])].tolist()
+            got.append((mem, int(grp.prefix_blocks[p])))
+        assert got == want, (trial, got, want)
+        for p, (mem, _) in enumerate(got):
+            for j, s in enumerate(mem):
+                assert int(grp.seq_prefix[s]) == p and int(grp.prefix_members[int(grp.seq_slot[s])]) == s
+        members = {s for mem, _ in got for s in mem}
+        assert all(int(grp.seq_prefix[s]) == -1 for s in range(n) if s not in members)

@@ -4,40 +4,54 @@ memory (no workspace: it uses a fixed scratch area built into the library).
 Runs last (file name), so a failure here cannot hide any other test.  It
 must pass alone in a fresh process and after the rest of the suite: the
 scratch area keeps the previous call's contents, so two calls in a row are
-checked against pa_decode with a caller workspace.
+checked against pa_decode with a caller workspace (the same kernels and the
+same split points, so the same bits) and against the CPU oracle.
 """
+import numpy as np
 import pytest
 import torch
 
 import pa_workloads as W
 import paged_kv_cache_452_b200 as pa
+from oracle.workload import expected
 from paged_kv_cache_452_b200 import runner
 
 pytestmark = pytest.mark.gpu
 
 TOL = {"bf16": 2e-2, "e4m3": 6e-2, "f32": 1e-4}
 
+CASES = {
+    "gqa_bf16": None, "fp8_long": None, "prefix_bf16": None,
+    # group 8 over 6016 tiles: the largest partial slots, contexts cut at
+    # many warp-range edges (still within the 8 MiB area)
+    "group8": dict(context_lens=[3000] * 16, num_q_heads=16, num_kv_heads=2),
+    # the CUDA-core path: fp32, and bf16 with a GQA group of 1
+    "tiny_fp32": None,
+    "mha_bf16": dict(context_lens=[7, 100, 0, 33], num_q_heads=4, num_kv_heads=4),
+}
 
-# group 8 over 6016 tiles: the largest partial slots, contexts cut at many
-# warp-range edges (still within the 8 MiB area)
-GROUP8 = dict(context_lens=[3000] * 16, num_q_heads=16, num_kv_heads=2)
+
+def _bits(t):
+    return t.detach().cpu().contiguous().view(torch.int32 if t.dtype == torch.float32 else torch.int16)
 
 
-@pytest.mark.parametrize("name", ["gqa_bf16", "fp8_long", "prefix_bf16", "group8"])
-def test_static_scratch_matches_workspace_path(name, cuda_device):
-    wl = W.custom(name, **GROUP8) if name == "group8" else W.make(name, "small")
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_static_scratch_matches_workspace_path_and_oracle(name, cuda_device):
+    kw = CASES[name]
+    wl = W.custom(name, **kw) if kw else W.make(name, "small")
     b = runner.setup(wl, cuda_device)
     runner.step(b)  # pa_cache_write + pa_decode with a caller workspace
     torch.cuda.synchronize()
-    ref = b.out.detach().clone().float()
     assert pa.workspace_error(b.workspace) == 0
+    ref = _bits(b.out)
+    exp = expected(wl)
     for _ in range(2):  # the second call finds the first one's scratch contents
         b.out.fill_(float("nan"))
         pa.pa_decode_static(b.desc, b.q, b.k_cache, b.v_cache, b.tables, b.seq_lens, b.scale, b.out)
         torch.cuda.synchronize()
-        got = b.out.detach().float()
-        assert torch.isfinite(got).all()
-        err = float((got - ref).abs().max())
+        assert torch.equal(_bits(b.out), ref), "static scratch and caller workspace differ"
+        got = b.out.detach().cpu().double().numpy()[exp["rows"]]
+        err = float(np.abs(got - exp["out"]).max())
         assert err <= TOL[wl.kv_dtype], err
 
 
