@@ -167,7 +167,9 @@ size_t pa_decode_workspace_size(const pa_cache_desc* desc, int32_t num_seqs);
  *               Its first 4 bytes are an error word the kernels set (never
  *               clear): 1 = a bounded internal wait timed out, 2 = a block
  *               table entry outside [0, num_blocks) (read as block 0),
- *               3 = a sequence longer than its table row (clamped).  Read it
+ *               3 = a sequence longer than its table row (clamped),
+ *               5 = an internal consistency check failed (a library bug;
+ *               the affected rows are not written).  Read it
  *               after the stream synchronises; after any error, zero the
  *               whole workspace again.  Calls sharing a workspace must not
  *               overlap on the GPU.  Bytes 4..7 are a fault-injection word

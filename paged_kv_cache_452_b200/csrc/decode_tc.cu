@@ -49,6 +49,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kGPad = 8;         // query rows per MMA N tile
 constexpr int kMaxStagesPerWarp = 8;
 constexpr int kSmemPerSM = 233472;  // B200: 228 KB per SM
+constexpr float kRefSlack = 8.f;    // log2 growth of a column max before its softmax reference moves
 // CTAs per SM: three (12 warps), as long as each warp's ring keeps two
 // stages; more warps hide the latency of the per-tile work (the e4m3
 // unpacking above all) and cut the tile space finer.  Measured against two
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
         atomicCAS(p.ws.err, 0, 2);
         d.blk = 0;
       }
-      if (i == 0 || t == wbeg) {
+      if (i == skip || t == wbeg) {  // the tile opens a piece
         d.row = p.rows.qsl ? __ldg(p.rows.qsl + s) : s;
         d.len = min(__ldg(p.rows.seq_lens + s), (nb + skip) * BS);
       }
@@ -439,6 +440,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
         const int4 inf = info[stage];
         row = inf.x;
         len = inf.y;
+        // the row comes from this warp's own bookkeeping; a value outside
+        // the batch is an internal inconsistency: flag it, write nothing
+        if ((unsigned)row >= (unsigned)p.rows.num_rows || len <= 0) {
+          if (lane == 0) atomicCAS(p.ws.err, 0, 5);
+          ok = false;
+          break;
+        }
         // ---- query fragments (B operand of S^T = K Q^T), rows >= G are zero ----
         const uint8_t* qs = ring + (size_t)stage * STAGE + C::KVB + g * D * 2;
         if constexpr (!C::FP8) {
@@ -548,16 +556,33 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
       }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float al0 = dev::ex2(m0 - mn0), al1 = dev::ex2(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
+      // Each column's exponentials use a reference that moves only when the
+      // column's max exceeds it by more than 2^8 (log2 units): then the
+      // running output and sum are rescaled; otherwise P = 2^(s - ref) stays
+      // at most 2^8 and nothing is rescaled.  Any reference gives the same
+      // result, and partials carry theirs as their max.
+      const bool mv0 = mx0 > m0 + kRefSlack, mv1 = mx1 > m1 + kRefSlack;
+      if (__any_sync(0xffffffffu, mv0 || mv1)) {
+        const float mn0 = mv0 ? mx0 : m0, mn1 = mv1 ? mx1 : m1;
+        const float al0 = dev::ex2(m0 - mn0), al1 = dev::ex2(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        l0 *= al0;
+        l1 *= al1;
+#pragma unroll
+        for (int i = 0; i < C::DM; ++i) {
+          o[i][0] *= al0;
+          o[i][1] *= al1;
+          o[i][2] *= al0;
+          o[i][3] *= al1;
+        }
+      }
       uint32_t pb0[C::KM], pb1[C::KM];
       float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
       for (int km = 0; km < C::KM; ++km) {
-        const float p00 = dev::ex2(sc[km][0] - mn0), p01 = dev::ex2(sc[km][1] - mn1);
-        const float p10 = dev::ex2(sc[km][2] - mn0), p11 = dev::ex2(sc[km][3] - mn1);
+        const float p00 = dev::ex2(sc[km][0] - m0), p01 = dev::ex2(sc[km][1] - m1);
+        const float p10 = dev::ex2(sc[km][2] - m0), p11 = dev::ex2(sc[km][3] - m1);
         ps0 += p00 + p10;
         ps1 += p01 + p11;
         if constexpr (C::FP8) {
@@ -568,15 +593,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
           pb1[km] = dev::movmatrix_t(dev::pack_bf16(p10, p11));
         }
       }
-      l0 = l0 * al0 + ps0;
-      l1 = l1 * al1 + ps1;
-#pragma unroll
-      for (int i = 0; i < C::DM; ++i) {
-        o[i][0] *= al0;
-        o[i][1] *= al1;
-        o[i][2] *= al0;
-        o[i][3] *= al1;
-      }
+      l0 += ps0;
+      l1 += ps1;
 
       // ---- O^T += V^T P^T ----
       if constexpr (!C::FP8) {
