@@ -75,7 +75,7 @@ struct Cfg {
 };
 
 struct SmemLayout {
-  uint32_t ring, bars, info, prefix, skip, total;
+  uint32_t ring, bars, info, prefix, total;
 };
 
 // A stage holds one tile's K and V and, when the tile opens a (sequence, kv
@@ -83,9 +83,7 @@ struct SmemLayout {
 // the next stage's tiles stay 1 KB aligned for the 128-byte swizzle).
 __host__ __device__ inline int q_area_bytes(int group, int d) { return (group * d * 2 + 1023) / 1024 * 1024; }
 
-// pfx: shared prefixes are skipped, so each sequence's skipped block count
-// is kept next to the tile prefix
-__host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int num_seqs, bool pfx) {
+__host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int num_seqs) {
   SmemLayout L;
   uint32_t off = 0;
   L.ring = off;
@@ -96,8 +94,6 @@ __host__ __device__ inline SmemLayout smem_layout(int stage_bytes, int nsw, int 
   off += (uint32_t)kWarps * nsw * 16;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
-  L.skip = off;
-  if (pfx) off += (uint32_t)num_seqs * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
   return L;
 }
@@ -128,6 +124,16 @@ __device__ __forceinline__ int cta_of(int x, int T, int P) { return (int)((((int
 // same order.
 __device__ __forceinline__ int kperm(int r) {
   return r < 8 ? 4 * (r >> 1) + (r & 1) : 4 * ((r - 8) >> 1) + 2 + (r & 1);
+}
+
+// Blocks of sequence s's row that its shared prefix covers (pa_decode_prefix;
+// 0 otherwise): the prefix kernel attends them, the decode skips them.  A
+// prefix that reaches the sequence's last token was refused in the
+// prologue (error 4), and such a sequence has no tiles.
+__device__ __forceinline__ int seq_skip(const DecodeParams& p, bool pfx, int s) {
+  if (!pfx) return 0;
+  const int pf = __ldg(p.pfx_of + s);
+  return pf >= 0 ? __ldg(p.pfx_blocks + pf) : 0;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -209,6 +215,67 @@ __device__ __forceinline__ void fused_write(const DecodeParams& p, uint8_t* st, 
   }
 }
 
+__device__ __forceinline__ void store_relaxed(int32_t* a, int32_t v) {
+  asm volatile("st.relaxed.gpu.global.s32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t load_relaxed(const int32_t* a) {
+  int32_t v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void prefetch_l2(const void* a, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(bytes) : "memory");
+}
+
+// Load balancing without moving work: a warp that has finished its range
+// looks at the published issue progress of 32 other warps per round (spread
+// over the grid), picks the one with the most tiles not yet issued and
+// prefetches up to 32 of that warp's last tiles (K and V) into L2.  The
+// owner's later TMA loads of those tiles then hit L2.  Stale or racing
+// progress values only make a prefetch useless, never wrong: every address
+// is recomputed from this launch's tile space and checked block ids.
+template <class C>
+__device__ __forceinline__ void help_prefetch(const DecodeParams& p, const int32_t* prefix, int S, int T, int W,
+                                              int wk, int lane) {
+  constexpr int BS = C::KM * 16;
+  constexpr int kRounds = 3;
+  const int hkv = p.num_kv_heads;
+  const bool pfx = p.pfx_of != nullptr;
+  for (int round = 0; round < kRounds; ++round) {
+    const int v = (int)(((int64_t)wk + 1 + (int64_t)(round * 32 + lane) * 53) % W);
+    const int vb = range_start(v, T, W), ve = range_start(v + 1, T, W);
+    const int prog = load_relaxed(p.ws.progress + v);
+    int left = (prog >= vb && prog < ve) ? ve - 1 - prog : 0;  // tiles v has not issued
+    int bv = v;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const int ol = __shfl_xor_sync(0xffffffffu, left, off), ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      if (ol > left || (ol == left && ov < bv)) {
+        left = ol;
+        bv = ov;
+      }
+    }
+    if (left < 2) return;  // no warp is far behind
+    // the victim's last `left` tiles, except the next one it is about to issue
+    const int vend = range_start(bv + 1, T, W);
+    const int t = vend - 1 - lane;
+    if (lane < left - 1) {
+      const int s = find_seq(prefix, S, hkv, t);
+      const int nb = prefix[s + 1] - prefix[s];
+      const int local = t - hkv * prefix[s];
+      const int h = local / nb;
+      const int i = local - h * nb + seq_skip(p, pfx, s);
+      const int blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + i);
+      if (blk >= 0 && blk < p.num_blocks) {
+        const int64_t off = ((int64_t)blk * hkv + h) * C::TILE;
+        prefetch_l2(p.k_cache + off, (uint32_t)C::TILE);
+        prefetch_l2(p.v_cache + off, (uint32_t)C::TILE);
+      }
+    }
+    __syncwarp();
+  }
+}
+
 template <int KV, int D, int BS>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -222,10 +289,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
   const int QA = q_area_bytes(G, D);
   const int STAGE = C::KVB + QA;  // bytes per ring stage
   const bool pfx = p.pfx_of != nullptr;
-  const SmemLayout L = smem_layout(STAGE, NSW, S, pfx);
+  const SmemLayout L = smem_layout(STAGE, NSW, S);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L.prefix);
-  // blocks of the sequence's row that a shared prefix covers (pa_decode_prefix)
-  int32_t* skipv = reinterpret_cast<int32_t*>(smem + L.skip);
   __shared__ int32_t warp_tot[kWarps];
 
   const int tid = threadIdx.x;
@@ -262,7 +327,6 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
           nb -= skip;
         }
       }
-      skipv[s] = skip;
     }
     prefix[s] = nb;
   }
@@ -339,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
       const int nb = prefix[s + 1] - prefix[s];
       const int local = t - hkv * prefix[s];
       d.h = local / nb;
-      const int skip = pfx ? skipv[s] : 0;
+      const int skip = seq_skip(p, pfx, s);
       const int i = local - d.h * nb + skip;
       d.blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + i);
       if (d.blk < 0 || d.blk >= p.num_blocks) {  // bad table entry: flag, read block 0
@@ -372,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     uint8_t* st = ring + (size_t)st_i * STAGE;
     const uint32_t qbytes = (uint32_t)(G * D * 2);
     if (lane == 0) {
+      store_relaxed(p.ws.progress + wk, wbeg + u);  // for warps that finish early (help_prefetch)
       if (rowj >= 0) info[st_i] = make_int4(rowj, lenj, 0, 0);
       dev::mbar_arrive_expect_tx(&full[st_i], (uint32_t)C::KVB + (rowj >= 0 ? qbytes : 0u));
     }
@@ -420,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     const int h = (t - seg0) / nb;
     const int a = seg0 + h * nb, b = a + nb;
     const int pe = min(b, wend);
-    const int skip = pfx ? skipv[s] : 0;  // tile a holds block `skip` of the row
+    const int skip = seq_skip(p, pfx, s);  // tile a holds block `skip` of the row
     int row = 0, len = 0;
     // this kv head's softmax and output scales (e4m3 per-head dequantisation)
     const float sl2 = p.k_head ? p.scale_log2 * __ldg(p.k_head + h) : p.scale_log2;
@@ -777,6 +842,12 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     }
     t = pe;
   }
+  if (ok) {
+    // this warp is done: pull the tiles other warps have not issued yet
+    // into L2, the furthest-behind warps first, so that their last loads hit
+    // L2.  Only a hint: no work moves and no result changes.
+    help_prefetch<C>(p, prefix, S, T, W, wk, lane);
+  }
   if (!ok && lane == 0) {
     // drain: let this warp's copies still in flight land before exiting
     for (int k = done; k < issued; ++k) dev::mbar_wait(&full[k % NSW], (uint32_t)((k / NSW) & 1), nullptr, 100000000ull);
@@ -793,8 +864,7 @@ template <int KV, int D, int BS>
 cudaError_t launch_instance(DecodeParams p, const CUtensorMap& tm_k, const CUtensorMap& tm_v, int num_sms,
                             cudaStream_t stream) {
   using C = Cfg<KV, D, BS>;
-  const SmemLayout L =
-      smem_layout(C::KVB + q_area_bytes(p.group, D), p.nstages, p.rows.num_seqs, p.pfx_of != nullptr);
+  const SmemLayout L = smem_layout(C::KVB + q_area_bytes(p.group, D), p.nstages, p.rows.num_seqs);
   auto kern = decode_tc_kernel<KV, D, BS>;
   // raise the kernel's dynamic shared memory limit once per device
   static int set_for[64] = {0};
@@ -837,19 +907,19 @@ cudaError_t launch_instance(DecodeParams p, const CUtensorMap& tm_k, const CUten
 
 int decode_tc_workers(int num_sms) { return kMaxCtasPerSM * num_sms * kWarps; }
 
-size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages, bool pfx) {
+size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages) {
   const int elem = kv == kFP8 ? 1 : 2;
   const int stage = 2 * block_size * head_dim * elem + q_area_bytes(group, head_dim);
-  return smem_layout(stage, nstages, num_seqs, pfx).total;
+  return smem_layout(stage, nstages, num_seqs).total;
 }
 
 // Ring stages per warp that fit `ctas` CTAs per SM.
-static int pick_stages(int kv, int head_dim, int block_size, int group, int num_seqs, bool pfx, int ctas) {
+static int pick_stages(int kv, int head_dim, int block_size, int group, int num_seqs, int ctas) {
   const int elem = kv == kFP8 ? 1 : 2;
   const int stage = 2 * block_size * head_dim * elem + q_area_bytes(group, head_dim);
   // 1 KB per CTA is reserved, plus a little static shared memory
   const int budget = kSmemPerSM / ctas - 1024 - 64;
-  const int fixed = (int)smem_layout(stage, 0, num_seqs, pfx).total;
+  const int fixed = (int)smem_layout(stage, 0, num_seqs).total;
   int n = (budget - fixed) / (kWarps * (stage + 8 + 16));
   if (n > kMaxStagesPerWarp) n = kMaxStagesPerWarp;
   return n;
@@ -861,6 +931,7 @@ size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int 
   off += ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;  // arrival counters
   off += (P * group * 2 * 4 + 255) / 256 * 256;                      // (max, sum)
   off += P * group * head_dim * 4;                                   // partial outputs
+  off += P * 4;                                                      // issue progress
   return off;
 }
 
@@ -871,7 +942,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p_in, const CUtensorMap& tm_k, 
   // ring, else fewer CTAs with deeper rings (large blocks)
   int ctas = kv == kFP8 ? ctas_per_sm<kFP8>() : ctas_per_sm<kBF16>();
   for (;; --ctas) {
-    p.nstages = pick_stages(kv, head_dim, block_size, p.group, p.rows.num_seqs, p.pfx_of != nullptr, ctas);
+    p.nstages = pick_stages(kv, head_dim, block_size, p.group, p.rows.num_seqs, ctas);
     if (p.nstages >= 2 || ctas == 1) break;
   }
   if (p.nstages < 2) return cudaErrorNotSupported;

@@ -54,11 +54,13 @@ struct DecodeWorkspace {
   unsigned int* cnt;        // [num_seqs * num_kv_heads] arrival counters: zero between calls
   float* ml;                // [workers][G][2] partial (max, sum), one cut piece per warp
   float* o;                 // [workers][G][D] partial unnormalised outputs
+  int32_t* progress;        // [workers] last tile each warp issued (a hint for idle warps; any value is safe)
 };
 
 struct DecodeParams {
   const uint8_t* q;  // bf16 [rows][Hq][D]
   uint8_t* out;      // bf16 [rows][Hq][D]
+  const uint8_t* k_cache;
   const uint8_t* v_cache;
   const int32_t* block_tables;
   int32_t max_blocks;
@@ -94,7 +96,7 @@ struct DecodeParams {
 // kv: kBF16 or kFP8; returns cudaErrorNotSupported for unsupported shapes.
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                              int kv, int head_dim, int block_size, int num_sms, cudaStream_t stream);
-size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages, bool pfx);
+size_t decode_tc_smem_bytes(int kv, int head_dim, int block_size, int group, int num_seqs, int nstages);
 int decode_tc_workers(int num_sms);  // the most worker warps a launch can have (workspace sizing)
 size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int head_dim, int num_sms);
 
