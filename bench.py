@@ -551,7 +551,7 @@ def bench_ours(args):
     cpu = cpu_baseline(wl, args.ref_budget) if (rank == 0 and not args.no_cpu_baseline) else None
     m.release()
 
-    per_config = {}
+    per_config = {wl.name: head}
     if not args.no_per_config:
         for name in PER_CONFIG:
             if name == wl.name:

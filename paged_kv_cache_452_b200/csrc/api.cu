@@ -180,8 +180,6 @@ WsCarve carve(void* base, int num_seqs, int num_kv_heads, int group, int head_di
   off += (P * group * 2 * 4 + 255) / 256 * 256;
   c.ws.o = reinterpret_cast<float*>(b + off);
   off += P * group * head_dim * 4;
-  c.ws.progress = reinterpret_cast<int32_t*>(b + off);
-  off += P * 4;
   c.bytes = off;
   return c;
 }
@@ -243,7 +241,6 @@ int run_decode_tc(const pa_cache_desc* d, const void* q, const void* k_cache, co
   DecodeParams p = {};
   p.q = static_cast<const uint8_t*>(q);
   p.out = static_cast<uint8_t*>(out);
-  p.k_cache = static_cast<const uint8_t*>(k_cache);
   p.v_cache = static_cast<const uint8_t*>(v_cache);
   p.block_tables = block_tables;
   p.max_blocks = max_blocks;
@@ -300,7 +297,6 @@ int run_simt(const pa_cache_desc* d, const void* q, const void* k_cache, const v
   p.err = static_cast<int32_t*>(workspace);
   p.q = static_cast<const uint8_t*>(q);
   p.out = static_cast<uint8_t*>(out);
-  p.k_cache = static_cast<const uint8_t*>(k_cache);
   p.v_cache = static_cast<const uint8_t*>(v_cache);
   p.block_tables = block_tables;
   p.max_blocks = max_blocks;

@@ -215,67 +215,6 @@ __device__ __forceinline__ void fused_write(const DecodeParams& p, uint8_t* st, 
   }
 }
 
-__device__ __forceinline__ void store_relaxed(int32_t* a, int32_t v) {
-  asm volatile("st.relaxed.gpu.global.s32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
-}
-__device__ __forceinline__ int32_t load_relaxed(const int32_t* a) {
-  int32_t v;
-  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ void prefetch_l2(const void* a, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(bytes) : "memory");
-}
-
-// Load balancing without moving work: a warp that has finished its range
-// looks at the published issue progress of 32 other warps per round (spread
-// over the grid), picks the one with the most tiles not yet issued and
-// prefetches up to 32 of that warp's last tiles (K and V) into L2.  The
-// owner's later TMA loads of those tiles then hit L2.  Stale or racing
-// progress values only make a prefetch useless, never wrong: every address
-// is recomputed from this launch's tile space and checked block ids.
-template <class C>
-__device__ __forceinline__ void help_prefetch(const DecodeParams& p, const int32_t* prefix, int S, int T, int W,
-                                              int wk, int lane) {
-  constexpr int BS = C::KM * 16;
-  constexpr int kRounds = 3;
-  const int hkv = p.num_kv_heads;
-  const bool pfx = p.pfx_of != nullptr;
-  for (int round = 0; round < kRounds; ++round) {
-    const int v = (int)(((int64_t)wk + 1 + (int64_t)(round * 32 + lane) * 53) % W);
-    const int vb = range_start(v, T, W), ve = range_start(v + 1, T, W);
-    const int prog = load_relaxed(p.ws.progress + v);
-    int left = (prog >= vb && prog < ve) ? ve - 1 - prog : 0;  // tiles v has not issued
-    int bv = v;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const int ol = __shfl_xor_sync(0xffffffffu, left, off), ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      if (ol > left || (ol == left && ov < bv)) {
-        left = ol;
-        bv = ov;
-      }
-    }
-    if (left < 2) return;  // no warp is far behind
-    // the victim's last `left` tiles, except the next one it is about to issue
-    const int vend = range_start(bv + 1, T, W);
-    const int t = vend - 1 - lane;
-    if (lane < left - 1) {
-      const int s = find_seq(prefix, S, hkv, t);
-      const int nb = prefix[s + 1] - prefix[s];
-      const int local = t - hkv * prefix[s];
-      const int h = local / nb;
-      const int i = local - h * nb + seq_skip(p, pfx, s);
-      const int blk = __ldg(p.block_tables + (int64_t)s * p.max_blocks + i);
-      if (blk >= 0 && blk < p.num_blocks) {
-        const int64_t off = ((int64_t)blk * hkv + h) * C::TILE;
-        prefetch_l2(p.k_cache + off, (uint32_t)C::TILE);
-        prefetch_l2(p.v_cache + off, (uint32_t)C::TILE);
-      }
-    }
-    __syncwarp();
-  }
-}
-
 template <int KV, int D, int BS>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -436,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     uint8_t* st = ring + (size_t)st_i * STAGE;
     const uint32_t qbytes = (uint32_t)(G * D * 2);
     if (lane == 0) {
-      store_relaxed(p.ws.progress + wk, wbeg + u);  // for warps that finish early (help_prefetch)
       if (rowj >= 0) info[st_i] = make_int4(rowj, lenj, 0, 0);
       dev::mbar_arrive_expect_tx(&full[st_i], (uint32_t)C::KVB + (rowj >= 0 ? qbytes : 0u));
     }
@@ -511,6 +449,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
           if (lane == 0) atomicCAS(p.ws.err, 0, 5);
           ok = false;
           break;
+        }
+        if (p.k_new != nullptr && pe == b && lane < 2 * (D * 2 / 128)) {
+          // pa_decode_fused: this piece ends the sequence, whose new K/V rows
+          // its last tile stores; pull them into L2 now so that the write
+          // does not wait on a cold load
+          const uint8_t* src = ((lane & 1) ? p.v_new : p.k_new) + ((int64_t)row * hkv + h) * D * 2 + (lane >> 1) * 128;
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
         }
         // ---- query fragments (B operand of S^T = K Q^T), rows >= G are zero ----
         const uint8_t* qs = ring + (size_t)stage * STAGE + C::KVB + g * D * 2;
@@ -842,12 +787,6 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
     }
     t = pe;
   }
-  if (ok) {
-    // this warp is done: pull the tiles other warps have not issued yet
-    // into L2, the furthest-behind warps first, so that their last loads hit
-    // L2.  Only a hint: no work moves and no result changes.
-    help_prefetch<C>(p, prefix, S, T, W, wk, lane);
-  }
   if (!ok && lane == 0) {
     // drain: let this warp's copies still in flight land before exiting
     for (int k = done; k < issued; ++k) dev::mbar_wait(&full[k % NSW], (uint32_t)((k / NSW) & 1), nullptr, 100000000ull);
@@ -931,7 +870,6 @@ size_t decode_tc_workspace_bytes(int num_seqs, int num_kv_heads, int group, int 
   off += ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;  // arrival counters
   off += (P * group * 2 * 4 + 255) / 256 * 256;                      // (max, sum)
   off += P * group * head_dim * 4;                                   // partial outputs
-  off += P * 4;                                                      // issue progress
   return off;
 }
 

@@ -54,13 +54,11 @@ struct DecodeWorkspace {
   unsigned int* cnt;        // [num_seqs * num_kv_heads] arrival counters: zero between calls
   float* ml;                // [workers][G][2] partial (max, sum), one cut piece per warp
   float* o;                 // [workers][G][D] partial unnormalised outputs
-  int32_t* progress;        // [workers] last tile each warp issued (a hint for idle warps; any value is safe)
 };
 
 struct DecodeParams {
   const uint8_t* q;  // bf16 [rows][Hq][D]
   uint8_t* out;      // bf16 [rows][Hq][D]
-  const uint8_t* k_cache;
   const uint8_t* v_cache;
   const int32_t* block_tables;
   int32_t max_blocks;
