@@ -297,6 +297,7 @@ int run_simt(const pa_cache_desc* d, const void* q, const void* k_cache, const v
   p.err = static_cast<int32_t*>(workspace);
   p.q = static_cast<const uint8_t*>(q);
   p.out = static_cast<uint8_t*>(out);
+  p.k_cache = static_cast<const uint8_t*>(k_cache);
   p.v_cache = static_cast<const uint8_t*>(v_cache);
   p.block_tables = block_tables;
   p.max_blocks = max_blocks;
