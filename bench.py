@@ -36,11 +36,18 @@ DEFAULT_WORKLOAD = "gqa_bf16"
 # profiled (keyed by its sha256): any edit to the source drops the figure to
 # null until the kernel is captured again.
 PROFILED_TRAFFIC = {
+    # mean of two captured launches
     "gqa_bf16": {"source": "paged_kv_cache_452_b200/csrc/decode_tc.cu",
-                 # the captured source with its header comment's CTA count corrected
-                 # (a comment-only edit, same line count; the code is unchanged)
-                 "sha256": "faab74a6d10b8ea93dd8d701d95eb0efa43c2f4d3fba534abb49367ada175fa1",
-                 "bytes": 294_643_200},
+                 "sha256": "974cd2f37d389fa5bd9de2254eda081369ece4b9165e537505fa2adc35ec77a3",
+                 "bytes": 294_879_232},
+    # captured on the first 16 of fp8_long's 128 sequences (the full pools are
+    # too large for a multi-pass capture) and scaled by the algorithmic bytes
+    "fp8_long": {"source": "paged_kv_cache_452_b200/csrc/decode_tc.cu",
+                 "sha256": "974cd2f37d389fa5bd9de2254eda081369ece4b9165e537505fa2adc35ec77a3",
+                 "bytes": 4_872_845_888},
+    "prefix_bf16": {"source": "paged_kv_cache_452_b200/csrc/decode_tc.cu",
+                    "sha256": "974cd2f37d389fa5bd9de2254eda081369ece4b9165e537505fa2adc35ec77a3",
+                    "bytes": 925_355_008},
     # mean of two captured launches
     "block_copy": {"source": "paged_kv_cache_452_b200/csrc/block_copy.cu",
                    "sha256": "14c4d4e16d7a6cfba5f9139645ec9d67aba270f8986a597db740b32a1a2c0f11",
@@ -412,7 +419,7 @@ class Measured:
              "step_gbs": job_throughput(world, self.alg_bytes, self.ms),
              "tokens_per_s": world * rows / (self.ms * 1e-3),
              "decode_tokens_per_s": world * decode_rows / (self.ms * 1e-3),
-             "clocks": self.clocks}
+             "clocks": self.clocks, "traffic": profiled_traffic(wl.name)}
         if self.fused_ms is not None:  # write + attention in one launch
             d["fused_step_us"] = self.fused_ms * 1e3
             d["fused_step_gbs"] = job_throughput(world, self.alg_bytes, self.fused_ms)
