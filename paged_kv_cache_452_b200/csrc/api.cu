@@ -519,6 +519,8 @@ int pa_decode_prefix(const pa_cache_desc* d, const void* q, const void* k_cache,
   pp.num_blocks = d->num_blocks;
   pp.scale_log2 = scale * 1.4426950408889634f;
   pp.err = static_cast<int32_t*>(workspace);
+  pp.unit_ctr = static_cast<int32_t*>(workspace) + 2;
+  pp.unit_exit = static_cast<int32_t*>(workspace) + 3;
   pp.pfx_start = prefix_start;
   pp.pfx_members = prefix_members;
   pp.pfx_blocks = prefix_blocks;
@@ -583,6 +585,9 @@ int pa_decode_chunked_prefill(const pa_cache_desc* d, const void* q, const void*
       pp.num_blocks = d->num_blocks;
       pp.scale_log2 = scale * 1.4426950408889634f;
       pp.err = static_cast<int32_t*>(workspace);
+      pp.unit_ctr = static_cast<int32_t*>(workspace) + 2;
+      pp.unit_exit = static_cast<int32_t*>(workspace) + 3;
+      pp.after_decode = 1;  // run_decode_tc launched this step's decode just before
       cudaError_t e = cudaErrorNotSupported;
       int sms = 0;
       if ((rc = num_sms(&sms))) return rc;

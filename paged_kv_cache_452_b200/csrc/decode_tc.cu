@@ -311,9 +311,14 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
         reinterpret_cast<__nv_bfloat16*>(p.out)[(int64_t)row * hq * D + i] = __float2bfloat16_rn(0.f);
     }
   }
-  dev::grid_dep_launch();
   const int wbeg = range_start(wk, T, W), wend = range_start(wk + 1, T, W);
-  if (wbeg >= wend) return;  // no CTA-wide synchronisation follows
+  if (wbeg >= wend) {
+    // no tiles: leave once the step's cache write is complete, so that a
+    // kernel launched behind this one (the step's prompt rows) can rely on
+    // every CTA of this grid having waited for it
+    dev::grid_dep_wait();
+    return;  // no CTA-wide synchronisation follows
+  }
 
   // ---- this warp's tiles: [wbeg, wend); warp-tile u is tile wbeg + u --------
   const int nmine = wend - wbeg;
@@ -399,6 +404,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<KV>())
   };
   int issued = 0;
   dev::grid_dep_wait();  // the pool rows this step wrote are visible from here on
+  // only now may a dependent launch start (it relies on this wait, above)
+  dev::grid_dep_launch();
   // Fault injection for tests (the workspace's second word, zero in normal
   // use): the later pieces of a cut context skip their count-in, so the
   // merging warp's wait runs out, after 1 ms instead of 2 s, and reports it.

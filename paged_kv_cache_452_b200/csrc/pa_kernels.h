@@ -110,6 +110,11 @@ struct PrefillParams {
   int32_t nstages_v;  // the tcgen05 kernel's V stages
   float scale_log2;
   int32_t* err;  // workspace error word
+  // the tcgen05 kernel's unit queue: a claim counter and a count of CTAs
+  // done, both zero between launches (workspace header words 2 and 3)
+  int32_t* unit_ctr;
+  int32_t* unit_exit;
+  int32_t after_decode;  // 1: launched right behind this step's decode kernel
   // Shared-prefix mode of the tcgen05 kernel (pa_decode_prefix): units are
   // (prefix, kv head, tile of members, chunk of prefix keys) and each writes
   // partial (max reference, sum, unnormalised O) rows instead of outputs.

@@ -51,6 +51,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemOptIn = 232448;  // 227 KB per block
 constexpr int kChunk = 128 * 128;   // one 128-byte-wide chunk of a 128-row tile
 constexpr float kRefSlack = 8.f;    // log2 growth of a row max before its reference moves
+constexpr int kUQ = 4;              // unit queue entries (the K loader claims, the other roles follow)
+// roles that read each queue entry: the V loader, the MMA thread and one
+// warp of each of the four row-warp pairs
+constexpr int kUQReaders = 6;
 
 template <int D, int BS>
 struct U {
@@ -66,7 +70,8 @@ struct U {
 
 struct Bars {
   // kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], then s_full[2],
-  // s_free[2], p_full, o_full, q_full, o_free, done
+  // s_free[2], p_full, o_full, q_full, o_free, done, uq_full[kUQ],
+  // uq_empty[kUQ]
   uint64_t* kfull;
   uint64_t* kempty;
   uint64_t* vfull;
@@ -78,10 +83,12 @@ struct Bars {
   uint64_t* q_full;
   uint64_t* o_free;
   uint64_t* done;
+  uint64_t* uq_full;
+  uint64_t* uq_empty;
 };
 
 struct ULayout {
-  uint32_t q, p, kring, vring, bars, tmem, xch, prefix, total;
+  uint32_t q, p, kring, vring, bars, tmem, uq, xch, prefix, total;
 };
 __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int nsv, int num_seqs) {
   ULayout L;
@@ -95,9 +102,11 @@ __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int ns
   L.vring = off;
   off += (uint32_t)kvt * nsv;
   L.bars = off;
-  off += (uint32_t)(2 * nsk + 2 * nsv + 9) * 8;
+  off += (uint32_t)(2 * nsk + 2 * nsv + 9 + 2 * kUQ) * 8;
   L.tmem = off;
   off += 16;
+  L.uq = off;  // unit queue [kUQ], then the row pairs' unit slots [4 quarters][2]
+  off += (kUQ + 8) * 4;
   L.xch = off;  // row max halves [2 tile parities][2 halves][128 rows], row sum halves [2][128]
   off += (2 * 2 * 128 + 2 * 128) * 4;
   L.prefix = off;
@@ -129,7 +138,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* vring = smem + L.vring;
   uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* bx = bar0 + 2 * NSK + 2 * NSV;
-  Bars B{bar0, bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 5, bx + 6, bx + 7, bx + 8};
+  Bars B{bar0, bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 5, bx + 6, bx + 7, bx + 8,
+         bx + 9, bx + 9 + kUQ};
+  int32_t* uq = reinterpret_cast<int32_t*>(smem + L.uq);
+  int32_t* pair_idx = uq + kUQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L.prefix);  // units before sequence s
   __shared__ int32_t warp_tot[kThreads / 32];
@@ -137,7 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = p.group, hq = p.num_q_heads, hkv = p.num_kv_heads;
   const int QB = kRows / G;  // query positions per unit
 
-  dev::grid_dep_wait();
+  // Launched right behind the decode kernel of the same step, this grid starts
+  // only once every decode CTA has passed its own wait for the step's cache
+  // write (it triggers its dependents after that wait), and its CTAs take SMs
+  // as the decode's CTAs leave them; it does not wait for the decode grid to
+  // finish, which it does not depend on.
+  if (!p.after_decode) dev::grid_dep_wait();
   // ---- units per prompt sequence (per prefix), exclusive prefix ---------------
   for (int s = tid; s < S; s += kThreads) {
     if constexpr (PFX) {
@@ -175,11 +192,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   dev::grid_dep_launch();
   const int nunits = prefix[S] * hkv;
-  if ((int)blockIdx.x >= nunits) return;  // nothing allocated yet
+  // Units are claimed from a counter in the workspace, in ordinal order, so a
+  // CTA that starts late or has short units simply takes fewer.  The last CTA
+  // to finish puts the counter back to zero for the next launch.
+  auto finish_queue = [&]() {
+    if (tid == 0) {
+      __threadfence();
+      if (atomicAdd(p.unit_exit, 1) == (int)gridDim.x - 1) {
+        atomicExch(p.unit_ctr, 0);
+        atomicExch(p.unit_exit, 0);
+      }
+    }
+  };
+  if ((int)blockIdx.x >= nunits) {  // nothing allocated yet
+    finish_queue();
+    return;
+  }
 
-  // Units are processed persistently: this CTA takes ordinals blockIdx.x,
-  // blockIdx.x + gridDim.x, ...  Ordinal i is query block i / Hkv (a
-  // sequence's last query blocks first) of kv head i % Hkv.
+  // Ordinal i is query block i / Hkv (a sequence's last query blocks first,
+  // the longest units of a sequence first) of kv head i % Hkv.
   // A unit's rows are query rows first + q0 .. first + q0 + qn - 1 (in PFX
   // mode: member slots first .. first + qn - 1); its keys are blocks
   // blk0 .. blk0 + nbneed - 1 of sequence s's table row.
@@ -251,6 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::mbar_init(B.q_full, kRowWarps);
     dev::mbar_init(B.o_free, kRowWarps);
     dev::mbar_init(B.done, 1);
+    for (int i = 0; i < kUQ; ++i) {
+      dev::mbar_init(&B.uq_full[i], 1);
+      dev::mbar_init(&B.uq_empty[i], kUQReaders);
+    }
     dev::fence_barrier_init();
   }
   if (warp == 1) {
@@ -286,7 +321,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     bool ok = true;
     int g = 0;
-    for (int idx = blockIdx.x; idx < nunits && ok; idx += gridDim.x) {
+    for (int n = 0;; ++n) {
+      // queue entry n: the K loader claims the unit and publishes it, the V
+      // loader reads it (a timed-out wait ends the walk, -1 for the others)
+      const int slot = n % kUQ;
+      int idx = -1;
+      if (!is_v) {
+        if (ok && lane == 0) idx = atomicAdd(p.unit_ctr, 1);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx >= nunits) idx = -1;
+        if (n >= kUQ && ok)
+          ok = __all_sync(0xffffffffu, dev::mbar_wait(&B.uq_empty[slot], (uint32_t)(((n / kUQ) - 1) & 1), p.err));
+        if (!ok) idx = -1;
+        if (lane == 0) {
+          uq[slot] = idx;
+          dev::mbar_arrive(&B.uq_full[slot]);
+        }
+      } else {
+        if (ok) ok = __all_sync(0xffffffffu, dev::mbar_wait(&B.uq_full[slot], (uint32_t)((n / kUQ) & 1), p.err));
+        if (ok) idx = uq[slot];
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&B.uq_empty[slot]);
+      }
+      __syncwarp();
+      if (idx < 0) break;
       const Unit u = unit_of(idx);
       int32_t enext = entry(u, 0);
       for (int k = 0; k < u.ntiles && ok; ++k, ++g) {
@@ -342,7 +400,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = true;
       int g0 = 0, nu = 0;  // first tile of the current unit; units done
-      for (int idx = blockIdx.x; idx < nunits && ok; idx += gridDim.x, ++nu) {
+      for (;; ++nu) {
+        const int slot = nu % kUQ;
+        int idx = -1;
+        if (ok) ok = dev::mbar_wait(&B.uq_full[slot], (uint32_t)((nu / kUQ) & 1), p.err);
+        if (ok) idx = uq[slot];
+        dev::mbar_arrive(&B.uq_empty[slot]);
+        if (idx < 0) break;
         const Unit u = unit_of(idx);
         ok = dev::mbar_wait(B.q_full, (uint32_t)(nu & 1), p.err);  // this unit's Q rows are in place
         if (ok && u.ntiles > 0) ok = issue_s(g0);
@@ -393,7 +457,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, dev::mbar_wait(bar, parity, p.err));
     };
     int g0 = 0;
-    for (int idx = blockIdx.x; idx < nunits; idx += gridDim.x) {
+    for (int n = 0;; ++n) {
+      // the pair's first warp reads queue entry n and hands it to the other
+      // through shared memory (two slots, alternating); both leave together
+      {
+        const int slot = n % kUQ;
+        if (hh == 0) {
+          int idx = -1;
+          wait_ok(&B.uq_full[slot], (uint32_t)((n / kUQ) & 1));
+          if (ok) idx = uq[slot];
+          __syncwarp();
+          if (lane == 0) {
+            pair_idx[quarter * 2 + (n & 1)] = idx;
+            dev::mbar_arrive(&B.uq_empty[slot]);
+          }
+        }
+        dev::named_bar_sync(pair_bar, 64);
+      }
+      const int idx = pair_idx[quarter * 2 + (n & 1)];
+      if (idx < 0) break;
       const Unit u = unit_of(idx);
       const bool valid = r < u.qn * G;
       const int pos = u.pos0 + u.q0 + r / G;  // the row's position: keys <= pos
@@ -570,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::tc_fence_after();
     dev::tmem_dealloc(tbase, kTmemCols);
   }
+  finish_queue();
 }
 
 template <int D, int BS, bool PFX = false>

@@ -82,6 +82,8 @@ def run_and_check(wl, device, seqs=None):
     err = float(np.abs(out - exp["out"]).max()) if out.size else 0.0
     assert err <= TOL[wl.kv_dtype], f"{wl.name}: max abs error {err}"
     assert pa.workspace_error(b.workspace) == 0
+    # the tcgen05 kernel's unit queue (header words 2 and 3) is back at zero
+    assert b.workspace[:16].view(torch.int32)[2:4].tolist() == [0, 0]
     return b, err
 
 
