@@ -22,17 +22,18 @@
 //    entries are read one tile ahead;
 //  * warp 1 holds the TMEM allocation and, from one thread, issues
 //    S = Q K^T (M 128, N 128, K 16 steps; double-buffered S in TMEM) and
-//    O += P V (N = head_dim; O stays in TMEM across tiles), committing each
-//    to an mbarrier; PV of a tile goes out as soon as its P is written, the
-//    S two tiles ahead after it;
+//    O += P V (N = head_dim; O stays in TMEM across tiles; P read from
+//    TMEM), committing each to an mbarrier; PV of a tile goes out as soon as
+//    its P is written, the S two tiles ahead after it;
 //  * warps 2..9 own half a query row per thread (two warps per TMEM lane
 //    quarter, so two per SM sub-partition): they read their 64 keys of the
 //    row of S from TMEM, mask (causal, context length), combine the row's max
 //    with the other half through shared memory, keep a running max reference that
 //    moves only when the row's max grows by more than 2^8 (then the row of
 //    O in TMEM and the running sum are rescaled: the result is unchanged,
-//    the rescale is rare), write P = 2^(s - ref) as bf16 into a swizzled
-//    shared tile for the PV MMA, and at the end divide O by the sum.
+//    the rescale is rare), write P = 2^(s - ref) as bf16 into one of two P
+//    buffers in TMEM (so a tile's softmax need not wait for the previous
+//    tile's PV to finish reading its P), and at the end divide O by the sum.
 // Every wait is bounded (2 s, then the error word is set); TMEM is freed on
 // every path.
 #include <cuda_runtime.h>
@@ -70,7 +71,7 @@ struct U {
 
 struct Bars {
   // kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], then s_full[2],
-  // s_free[2], p_full, o_full, q_full, o_free, done, uq_full[kUQ],
+  // s_free[2], p_full[2], o_full[2], q_full, o_free, done, uq_full[kUQ],
   // uq_empty[kUQ]
   uint64_t* kfull;
   uint64_t* kempty;
@@ -88,21 +89,19 @@ struct Bars {
 };
 
 struct ULayout {
-  uint32_t q, p, kring, vring, bars, tmem, uq, xch, prefix, total;
+  uint32_t q, kring, vring, bars, tmem, uq, xch, prefix, total;
 };
 __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int nsv, int num_seqs) {
   ULayout L;
   uint32_t off = 0;
   L.q = off;
   off += qbytes;
-  L.p = off;
-  off += 2 * kChunk;
   L.kring = off;
   off += (uint32_t)kvt * nsk;
   L.vring = off;
   off += (uint32_t)kvt * nsv;
   L.bars = off;
-  off += (uint32_t)(2 * nsk + 2 * nsv + 9 + 2 * kUQ) * 8;
+  off += (uint32_t)(2 * nsk + 2 * nsv + 11 + 2 * kUQ) * 8;
   L.tmem = off;
   off += 16;
   L.uq = off;  // unit queue [kUQ], then the row pairs' unit slots [4 quarters][2]
@@ -133,13 +132,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int S = p.rows.num_seqs;
   const ULayout L = u_layout(C::QBYTES, C::KVT, NSK, NSV, S);
   uint8_t* qs = smem + L.q;
-  uint8_t* ps = smem + L.p;
   uint8_t* kring = smem + L.kring;
   uint8_t* vring = smem + L.vring;
   uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* bx = bar0 + 2 * NSK + 2 * NSV;
-  Bars B{bar0, bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 5, bx + 6, bx + 7, bx + 8,
-         bx + 9, bx + 9 + kUQ};
+  Bars B{bar0, bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 6, bx + 8, bx + 9, bx + 10,
+         bx + 11, bx + 11 + kUQ};
   int32_t* uq = reinterpret_cast<int32_t*>(smem + L.uq);
   int32_t* pair_idx = uq + kUQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem);
@@ -277,8 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&B.s_full[i], 1);
       dev::mbar_init(&B.s_free[i], kRowWarps);
     }
-    dev::mbar_init(B.p_full, kRowWarps);
-    dev::mbar_init(B.o_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      dev::mbar_init(&B.p_full[i], kRowWarps);
+      dev::mbar_init(&B.o_full[i], 1);
+    }
     dev::mbar_init(B.q_full, kRowWarps);
     dev::mbar_init(B.o_free, kRowWarps);
     dev::mbar_init(B.done, 1);
@@ -296,7 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   dev::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t t_s0 = tbase, t_o = tbase + 2 * kKeys;  // S buffers at columns 0 and 128, O at 256
+  // S buffers at columns 0 and 128, O at 256 (D columns), then the two P
+  // buffers (64 columns each: 128 bf16 keys per row)
+  const uint32_t t_s0 = tbase, t_o = tbase + 2 * kKeys, t_p = t_o + D;
+  static_assert(2 * kKeys + D + 2 * (kKeys / 2) <= (int)kTmemCols, "TMEM columns");
   // Tiles are counted over all of this CTA's units ("g"): ring stages,
   // S buffers and the per-tile barriers' phases follow that count.
 
@@ -380,7 +383,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors built once; an MMA adds its byte offset / 16 to the
       // start-address field (addresses stay below 256 KB: no carry out)
       const uint64_t dq = dev::umma_desc_sw128(dev::smem_u32(qs), 16, 1024);
-      const uint64_t dp = dev::umma_desc_sw128(dev::smem_u32(ps), 16, 1024);
       const uint64_t dk = dev::umma_desc_sw128(dev::smem_u32(kring), 16, 1024);
       const uint64_t dv = dev::umma_desc_sw128(dev::smem_u32(vring), kChunk, 1024);
       // S[g & 1] = Q K_g^T once K_g has landed and S[g & 1]'s last reader is done
@@ -413,7 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && u.ntiles > 1) ok = issue_s(g0 + 1);
         for (int k = 0; k < u.ntiles && ok; ++k) {
           const int g = g0 + k;
-          ok = dev::mbar_wait(B.p_full, (uint32_t)(g & 1), p.err) &&
+          // p_full[g & 1] and o_full[g & 1] complete once per tile of that
+          // parity: tile g is their phase g >> 1
+          ok = dev::mbar_wait(&B.p_full[g & 1], (uint32_t)((g >> 1) & 1), p.err) &&
                dev::mbar_wait(&B.vfull[g % NSV], (uint32_t)((g / NSV) & 1), p.err);
           // the previous unit's O has been read out before this unit overwrites it
           if (ok && k == 0 && nu > 0) ok = dev::mbar_wait(B.o_free, (uint32_t)((nu - 1) & 1), p.err);
@@ -422,12 +426,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t vb = dv + (uint64_t)(((g % NSV) * C::KVT) >> 4);
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS_O; ++ks) {
-            // A = P (K-major, 16 keys per step); B = V (MN-major: d contiguous,
-            // 64-wide chunks kChunk apart, 8-key row groups 1024 bytes apart)
-            const uint64_t aoff = (uint64_t)(((ks >> 2) * kChunk + (ks & 3) * 32) >> 4);
-            dev::umma_ss(t_o, dp + aoff, vb + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, (k > 0 || ks > 0) ? 1u : 0u);
+            // A = P from TMEM buffer g & 1 (16 keys = 8 columns per step); B =
+            // V (MN-major: d contiguous, 64-wide chunks kChunk apart, 8-key row
+            // groups 1024 bytes apart)
+            dev::umma_ts(t_o, t_p + (uint32_t)((g & 1) * (kKeys / 2) + 8 * ks),
+                         vb + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, (k > 0 || ks > 0) ? 1u : 0u);
           }
-          dev::umma_commit(B.o_full);
+          dev::umma_commit(&B.o_full[g & 1]);
           dev::umma_commit(&B.vempty[g % NSV]);
           if (k + 2 < u.ntiles) ok = issue_s(g + 2);
         }
@@ -550,11 +555,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[i] = dev::pack_bf16(a, b);
         }
         lsum += (sp[0] + sp[1]) + (sp[2] + sp[3]);
-        // the previous PV MMA has finished: P may be rewritten, O is stable
-        if (k > 0) {
-          wait_ok(B.o_full, (uint32_t)((g - 1) & 1));
+        // a rescale needs O stable: the previous tile's PV has finished
+        if (k > 0 && __any_sync(0xffffffffu, move)) {
+          wait_ok(&B.o_full[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1));
           dev::tc_fence_after();
-          if (__any_sync(0xffffffffu, move)) {
+          {
             // rescale this row's half of O in TMEM (rows that keep their
             // reference use 1)
 #pragma unroll 1
@@ -568,11 +573,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // this half's 64 keys are chunk hh of the swizzled P tile
-#pragma unroll
-        for (int uu = 0; uu < 8; ++uu)
-          *reinterpret_cast<uint4*>(ps + hh * kChunk + swz(r, uu)) =
-              make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+        // P buffer g & 1 was last read by the PV of tile g - 2 (an earlier
+        // unit's PVs are all done: its epilogue waited for them)
+        if (k >= 2) {
+          wait_ok(&B.o_full[g & 1], (uint32_t)(((g >> 1) - 1) & 1));
+          dev::tc_fence_after();
+        }
+        // this half's 64 keys, two per column, into P buffer g & 1
+        dev::tmem_st32(t_p + (uint32_t)((g & 1) * (kKeys / 2) + (kKeys / 4) * hh) + lane_addr, pk);
         // the tile holding the context's end: slots past it hold stale pool
         // bytes (masked scores, but 0 * NaN would poison P V): zero their V rows
         const int key0 = k * kKeys;
@@ -590,11 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         dev::tc_fence_before();
         __syncwarp();
-        if (lane == 0) dev::mbar_arrive(B.p_full);
+        if (lane == 0) dev::mbar_arrive(&B.p_full[g & 1]);
       }
       // ---- O / sum -> this half of the output row; then O is free ----
       if (u.ntiles > 0) {
-        wait_ok(B.o_full, (uint32_t)((g0 + u.ntiles - 1) & 1));
+        wait_ok(&B.o_full[(g0 + u.ntiles - 1) & 1], (uint32_t)(((g0 + u.ntiles - 1) >> 1) & 1));
         dev::tc_fence_after();
         xsum[hh * 128 + r] = lsum;
         dev::named_bar_sync(pair_bar, 64);
