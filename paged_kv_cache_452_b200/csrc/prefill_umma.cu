@@ -13,7 +13,7 @@
 // tile serves all of them.  One persistent CTA per SM walks its share of the
 // units; the rings, the S buffers and the barriers run on across units, so
 // the next unit's first tiles load while the current one finishes.
-//  * warps 0 and 10 walk the block table and bring the K and the V halves of
+//  * warps 0 and 18 walk the block table and bring the K and the V halves of
 //    128-key tiles into two rings of shared-memory stages with TMA (2-D
 //    boxes of [block][128 B], 128-byte swizzle, boxes of consecutive blocks
 //    stacked into one swizzled tile); a K stage is free again as soon as its
@@ -25,10 +25,11 @@
 //    O += P V (N = head_dim; O stays in TMEM across tiles; P read from
 //    TMEM), committing each to an mbarrier; PV of a tile goes out as soon as
 //    its P is written, the S two tiles ahead after it;
-//  * warps 2..9 own half a query row per thread (two warps per TMEM lane
-//    quarter, so two per SM sub-partition): they read their 64 keys of the
-//    row of S from TMEM, mask (causal, context length), combine the row's max
-//    with the other half through shared memory, keep a running max reference that
+//  * warps 2..17 own a quarter of a query row per thread (four warps per
+//    TMEM lane quarter, so four per SM sub-partition to hide each tile's
+//    latencies): they read their 32 keys of the row of S from TMEM, mask
+//    (causal, context length), combine the row's max with the other quarters
+//    through shared memory, keep a running max reference that
 //    moves only when the row's max grows by more than 2^8 (then the row of
 //    O in TMEM and the running sum are rescaled: the result is unchanged,
 //    the rescale is rare), write P = 2^(s - ref) as bf16 into one of two P
@@ -46,15 +47,20 @@ namespace {
 
 constexpr int kRows = 128;    // query rows per unit (positions x group): the MMA's M
 constexpr int kKeys = 128;    // keys per K/V tile: N of S = Q K^T, K of O = P V
-constexpr int kThreads = 352;  // warps 0/10 load K/V, warp 1 issues MMAs, warps 2..9 half a row per thread
-constexpr int kRowWarps = 8;
+// Each query row is split into kParts parts (kKeys / kParts keys of every
+// tile, D / kParts columns of O), one thread per part: four row warps per
+// TMEM lane quarter, so every SM sub-partition runs four softmax warps.
+constexpr int kParts = 4;
+constexpr int kRowWarps = 4 * kParts;
+constexpr int kThreads = 32 * (kRowWarps + 3);  // warp 0 loads K, warp 1 issues MMAs, then the row warps, last loads V
+constexpr int kVWarp = kRowWarps + 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemOptIn = 232448;  // 227 KB per block
 constexpr int kChunk = 128 * 128;   // one 128-byte-wide chunk of a 128-row tile
 constexpr float kRefSlack = 8.f;    // log2 growth of a row max before its reference moves
 constexpr int kUQ = 4;              // unit queue entries (the K loader claims, the other roles follow)
 // roles that read each queue entry: the V loader, the MMA thread and one
-// warp of each of the four row-warp pairs
+// warp of each of the four row-warp groups (one group per TMEM lane quarter)
 constexpr int kUQReaders = 6;
 
 template <int D, int BS>
@@ -104,10 +110,10 @@ __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int ns
   off += (uint32_t)(2 * nsk + 2 * nsv + 11 + 2 * kUQ) * 8;
   L.tmem = off;
   off += 16;
-  L.uq = off;  // unit queue [kUQ], then the row pairs' unit slots [4 quarters][2]
+  L.uq = off;  // unit queue [kUQ], then the row groups' unit slots [4 quarters][2]
   off += (kUQ + 8) * 4;
-  L.xch = off;  // row max halves [2 tile parities][2 halves][128 rows], row sum halves [2][128]
-  off += (2 * 2 * 128 + 2 * 128) * 4;
+  L.xch = off;  // row max parts [2 tile parities][kParts][128 rows], row sum parts [kParts][128]
+  off += (2 * kParts * 128 + kParts * 128) * 4;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
@@ -303,9 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Tiles are counted over all of this CTA's units ("g"): ring stages,
   // S buffers and the per-tile barriers' phases follow that count.
 
-  if (warp == 0 || warp == 10) {
-    // ======================= loads: the K (warp 0) or V (warp 10) ring ========
-    const bool is_v = warp == 10;
+  if (warp == 0 || warp == kVWarp) {
+    // ======================= loads: the K (warp 0) or V (last warp) ring ======
+    const bool is_v = warp == kVWarp;
     const int nsr = is_v ? NSV : NSK;
     uint64_t* fullb = is_v ? B.vfull : B.kfull;
     uint64_t* emptyb = is_v ? B.vempty : B.kempty;
@@ -445,26 +451,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ======================= rows: softmax, P, output =========================
-    // Thread = (row r, half hh): keys [64 hh, 64 hh + 64) of each tile and O
-    // columns [hh D/2, (hh+1) D/2).  The two warps of a lane quarter meet at
+    // Thread = (row r, part hh): keys [HK hh, HK (hh+1)) of each tile and O
+    // columns [HD hh, HD (hh+1)).  The kParts warps of a lane quarter meet at
     // named barrier 1 + quarter; they run the same units and tiles and pass
     // the same barriers even after a timed-out wait (then they skip the
-    // remaining waits), so neither can be left waiting.
-    constexpr int HK = kKeys / 2, HD = D / 2;
+    // remaining waits), so none can be left waiting.
+    constexpr int HK = kKeys / kParts, HD = D / kParts;
+    static_assert(HK == 32 && (HD == 32 || HD == 16), "one TMEM load of S per part, one or half of O");
     const int quarter = warp & 3, hh = (warp - 2) >> 2;
     const int r = 32 * quarter + lane;  // this thread's row (its TMEM lane)
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
     const int pair_bar = 1 + quarter;
-    float* xmax = reinterpret_cast<float*>(smem + L.xch);  // [tile parity][half][row]
-    float* xsum = xmax + 2 * 2 * 128;                       // [half][row]
+    constexpr int kGroup = 32 * kParts;                     // threads at a quarter's named barrier
+    float* xmax = reinterpret_cast<float*>(smem + L.xch);  // [tile parity][part][row]
+    float* xsum = xmax + 2 * kParts * 128;                  // [part][row]
     bool ok = true;
     auto wait_ok = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(0xffffffffu, dev::mbar_wait(bar, parity, p.err));
     };
     int g0 = 0;
     for (int n = 0;; ++n) {
-      // the pair's first warp reads queue entry n and hands it to the other
-      // through shared memory (two slots, alternating); both leave together
+      // the group's first warp reads queue entry n and hands it to the others
+      // through shared memory (two slots, alternating); all leave together
       {
         const int slot = n % kUQ;
         if (hh == 0) {
@@ -477,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dev::mbar_arrive(&B.uq_empty[slot]);
           }
         }
-        dev::named_bar_sync(pair_bar, 64);
+        dev::named_bar_sync(pair_bar, kGroup);
       }
       const int idx = pair_idx[quarter * 2 + (n & 1)];
       if (idx < 0) break;
@@ -488,13 +496,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // member slot first + r / G
       const int qrow = !PFX ? u.first + u.q0 + r / G : (valid ? __ldg(p.pfx_members + u.first + r / G) : 0);
       const int64_t grow = ((int64_t)qrow * hq + (int64_t)u.h * G + r % G) * D;
-      // ---- this half of the Q row into the swizzled Q tile (zero for rows
+      // ---- this part of the Q row into the swizzled Q tile (zero for rows
       // past the unit); the previous unit's MMAs have all completed (its
       // output was read after them)
       {
         const uint4* src = reinterpret_cast<const uint4*>(p.q + grow * 2);
+        constexpr int VU = C::NCH * 8 / kParts;  // 16-byte units of a part
 #pragma unroll
-        for (int v = hh * C::NCH * 4; v < (hh + 1) * C::NCH * 4; ++v) {
+        for (int v = hh * VU; v < (hh + 1) * VU; ++v) {
           const uint4 x = valid ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
           *reinterpret_cast<uint4*>(qs + (v >> 3) * kChunk + swz(r, v & 7)) = x;
         }
@@ -510,19 +519,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sv[HK];
         {
           uint32_t w[32];
+          dev::tmem_ld32(t_s0 + (uint32_t)((g & 1) * kKeys + HK * hh) + lane_addr, w);
 #pragma unroll
-          for (int c = 0; c < HK / 32; ++c) {
-            dev::tmem_ld32(t_s0 + (uint32_t)((g & 1) * kKeys + HK * hh + 32 * c) + lane_addr, w);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[32 * c + i] = __uint_as_float(w[i]);
-          }
+          for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(w[i]);
         }
         dev::tc_fence_before();
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(&B.s_free[g & 1]);
-        // mask; this half's max, then the row's (the scale is positive, so
+        // mask; this part's max, then the row's (the scale is positive, so
         // it is applied to the max and folded into the exponent's FMA)
-        const int lim = min(pos + 1, u.seq_len) - k * kKeys - HK * hh;  // keys [0, lim) of this half are visible
+        const int lim = min(pos + 1, u.seq_len) - k * kKeys - HK * hh;  // keys [0, lim) of this part are visible
         float mp[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) mp[i] = -INFINITY;
@@ -532,9 +538,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mp[i & 3] = fmaxf(mp[i & 3], sv[i]);
         }
         const float mh = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-        xmax[((g & 1) * 2 + hh) * 128 + r] = mh;
-        dev::named_bar_sync(pair_bar, 64);
-        const float mx = fmaxf(mh, xmax[((g & 1) * 2 + (hh ^ 1)) * 128 + r]) * p.scale_log2;
+        xmax[((g & 1) * kParts + hh) * 128 + r] = mh;
+        dev::named_bar_sync(pair_bar, kGroup);
+        float mrow = mh;
+#pragma unroll
+        for (int q2 = 0; q2 < kParts; ++q2) mrow = fmaxf(mrow, xmax[((g & 1) * kParts + q2) * 128 + r]);
+        const float mx = mrow * p.scale_log2;
         const bool move = mx > ref + kRefSlack;
         const float alpha = move ? dev::ex2(ref - mx) : 1.f;
         if (move) {
@@ -560,17 +569,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           wait_ok(&B.o_full[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1));
           dev::tc_fence_after();
           {
-            // rescale this row's half of O in TMEM (rows that keep their
+            // rescale this row's part of O in TMEM (rows that keep their
             // reference use 1)
-#pragma unroll 1
-            for (int c = 0; c < HD / 32; ++c) {
-              uint32_t w[32];
-              const uint32_t ta = t_o + (uint32_t)(HD * hh + 32 * c) + lane_addr;
-              dev::tmem_ld32(ta, w);
+            const uint32_t ta = t_o + (uint32_t)(HD * hh) + lane_addr;
+            uint32_t w[HD];
+            if constexpr (HD == 32) dev::tmem_ld32(ta, w); else dev::tmem_ld16(ta, w);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-              dev::tmem_st32(ta, w);
-            }
+            for (int i = 0; i < HD; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+            if constexpr (HD == 32) dev::tmem_st32(ta, w); else dev::tmem_st16(ta, w);
           }
         }
         // P buffer g & 1 was last read by the PV of tile g - 2 (an earlier
@@ -579,8 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           wait_ok(&B.o_full[g & 1], (uint32_t)(((g >> 1) - 1) & 1));
           dev::tc_fence_after();
         }
-        // this half's 64 keys, two per column, into P buffer g & 1
-        dev::tmem_st32(t_p + (uint32_t)((g & 1) * (kKeys / 2) + (kKeys / 4) * hh) + lane_addr, pk);
+        // this part's HK keys, two per column, into P buffer g & 1
+        dev::tmem_st16(t_p + (uint32_t)((g & 1) * (kKeys / 2) + (HK / 2) * hh) + lane_addr, pk);
         // the tile holding the context's end: slots past it hold stale pool
         // bytes (masked scores, but 0 * NaN would poison P V): zero their V rows
         const int key0 = k * kKeys;
@@ -600,50 +606,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(&B.p_full[g & 1]);
       }
-      // ---- O / sum -> this half of the output row; then O is free ----
+      // ---- O / sum -> this part of the output row; then O is free ----
       if (u.ntiles > 0) {
         wait_ok(&B.o_full[(g0 + u.ntiles - 1) & 1], (uint32_t)(((g0 + u.ntiles - 1) >> 1) & 1));
         dev::tc_fence_after();
         xsum[hh * 128 + r] = lsum;
-        dev::named_bar_sync(pair_bar, 64);
-        const float total = lsum + xsum[(hh ^ 1) * 128 + r];
+        dev::named_bar_sync(pair_bar, kGroup);
+        float total = 0.f;
+#pragma unroll
+        for (int q2 = 0; q2 < kParts; ++q2) total += xsum[q2 * 128 + r];
+        uint32_t w[HD];
+        if constexpr (HD == 32) dev::tmem_ld32(t_o + (uint32_t)(HD * hh) + lane_addr, w);
+        else dev::tmem_ld16(t_o + (uint32_t)(HD * hh) + lane_addr, w);
         if constexpr (PFX) {
           // partial row of member slot first + r / G, q head h * G + r % G:
-          // (max reference, sum) and this half of the unnormalised O
+          // (max reference, sum) and this part of the unnormalised O
           const int64_t prow =
               ((int64_t)u.chunk * p.num_members + u.first + r / G) * hq + (int64_t)u.h * G + r % G;
           if (valid && ok && hh == 0) *reinterpret_cast<float2*>(p.pfx_ml + prow * 2) = make_float2(ref, total);
           float4* dst = reinterpret_cast<float4*>(p.pfx_o + prow * D + HD * hh);
-#pragma unroll 1
-          for (int c = 0; c < HD / 32; ++c) {
-            uint32_t w[32];
-            dev::tmem_ld32(t_o + (uint32_t)(HD * hh + 32 * c) + lane_addr, w);
-            if (valid && ok) {
-#pragma unroll
-              for (int uu = 0; uu < 8; ++uu)
-                dst[8 * c + uu] = make_float4(__uint_as_float(w[4 * uu]), __uint_as_float(w[4 * uu + 1]),
-                                              __uint_as_float(w[4 * uu + 2]), __uint_as_float(w[4 * uu + 3]));
-            }
-          }
-        } else {
-        const float inv = valid ? 1.f / total : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (grow + HD * hh) * 2);
-#pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t w[32];
-          dev::tmem_ld32(t_o + (uint32_t)(HD * hh + 32 * c) + lane_addr, w);
           if (valid && ok) {
 #pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
+            for (int uu = 0; uu < HD / 4; ++uu)
+              dst[uu] = make_float4(__uint_as_float(w[4 * uu]), __uint_as_float(w[4 * uu + 1]),
+                                    __uint_as_float(w[4 * uu + 2]), __uint_as_float(w[4 * uu + 3]));
+          }
+        } else {
+          const float inv = valid ? 1.f / total : 0.f;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (grow + HD * hh) * 2);
+          if (valid && ok) {
+#pragma unroll
+            for (int uu = 0; uu < HD / 8; ++uu) {
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 pk[e] = dev::pack_bf16(__uint_as_float(w[8 * uu + 2 * e]) * inv,
                                        __uint_as_float(w[8 * uu + 2 * e + 1]) * inv);
-              dst[4 * c + uu] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[uu] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           }
-        }
         }
       }
       dev::tc_fence_before();
