@@ -23,8 +23,9 @@
 //  * warp 1 holds the TMEM allocation and, from one thread, issues
 //    S = Q K^T (M 128, N 128, K 16 steps; double-buffered S in TMEM) and
 //    O += P V (N = head_dim; O stays in TMEM across tiles; P read from
-//    TMEM), committing each to an mbarrier; PV of a tile goes out as soon as
-//    its P is written, the S two tiles ahead after it;
+//    TMEM), committing each to an mbarrier; the S two tiles ahead goes out
+//    as soon as the row warps have read a tile's S, its PV once its P is
+//    written;
 //  * warps 2..17 own a quarter of a query row per thread (four warps per
 //    TMEM lane quarter, so four per SM sub-partition to hide each tile's
 //    latencies): they read their 32 keys of the row of S from TMEM, mask
@@ -421,6 +422,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && u.ntiles > 1) ok = issue_s(g0 + 1);
         for (int k = 0; k < u.ntiles && ok; ++k) {
           const int g = g0 + k;
+          // S two tiles ahead goes out as soon as the row warps have read
+          // S_g out of its buffer (early in tile g's softmax), so it has two
+          // softmax durations to complete before they need it
+          if (k + 2 < u.ntiles) ok = issue_s(g + 2);
+          if (!ok) break;
           // p_full[g & 1] and o_full[g & 1] complete once per tile of that
           // parity: tile g is their phase g >> 1
           ok = dev::mbar_wait(&B.p_full[g & 1], (uint32_t)((g >> 1) & 1), p.err) &&
@@ -440,7 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           dev::umma_commit(&B.o_full[g & 1]);
           dev::umma_commit(&B.vempty[g % NSV]);
-          if (k + 2 < u.ntiles) ok = issue_s(g + 2);
         }
         g0 += u.ntiles;
       }
