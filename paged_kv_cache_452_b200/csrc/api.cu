@@ -157,6 +157,27 @@ int encode_kv_map(CUtensorMap* m, const void* base, int dt, const pa_cache_desc*
   return PA_OK;
 }
 
+// 3-D map over the queries [tokens][Hq][D] (bf16) for the tcgen05 prompt-row
+// kernel: a box is [128 / G tokens][G heads][64 elements], 128-byte swizzle,
+// so one box fills one 64-column chunk of a unit's Q tile in row order
+// (position-major, group head minor).
+int encode_q_map(CUtensorMap* m, const void* q, int num_tokens, const pa_cache_desc* d) {
+  auto enc = encode_fn();
+  if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const int group = d->num_q_heads / d->num_kv_heads;
+  cuuint64_t dims[3] = {(cuuint64_t)d->head_dim, (cuuint64_t)d->num_q_heads, (cuuint64_t)num_tokens};
+  // each stride steps over the whole previous dimension: rows do not overlap
+  cuuint64_t strides[2] = {(cuuint64_t)d->head_dim * 2, (cuuint64_t)d->num_q_heads * d->head_dim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (!aligned(q, 16)) return fail(PA_ERR_INVALID_ARG, "q must be 16-byte aligned");
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return PA_OK;
+}
+
 int cuda_status(cudaError_t e, const char* who) {
   if (e == cudaSuccess) return PA_OK;
   return fail(PA_ERR_CUDA, "%s: %s", who, cudaGetErrorString(e));
@@ -591,7 +612,11 @@ int pa_decode_chunked_prefill(const pa_cache_desc* d, const void* q, const void*
       cudaError_t e = cudaErrorNotSupported;
       int sms = 0;
       if ((rc = num_sms(&sms))) return rc;
-      if (umma) e = launch_prefill_umma(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, sms, st);
+      if (umma) {
+        CUtensorMap tm_q;
+        if ((rc = encode_q_map(&tm_q, q, num_tokens, d))) return rc;
+        e = launch_prefill_umma(pp, tm_k, tm_v, tm_q, d->head_dim, d->block_size, num_tokens, sms, st);
+      }
       if (e == cudaErrorNotSupported && prefill_tc_supported(d->kv_dtype, d->q_dtype, d->head_dim, d->block_size, group))
         e = launch_prefill_tc(pp, tm_k, tm_v, d->head_dim, d->block_size, num_tokens, st);
       if (e != cudaErrorNotSupported) return cuda_status(e, who);

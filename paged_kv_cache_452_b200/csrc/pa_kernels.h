@@ -136,8 +136,12 @@ bool prefill_tc_supported(int kv, int q, int head_dim, int block_size, int group
 // The same rows on tcgen05 (TMEM accumulators); cudaErrorNotSupported when
 // the shape or the batch's unit table does not fit (the caller falls back).
 bool prefill_umma_supported(int kv, int q, int head_dim, int block_size, int group);
+// tm_q: the queries as [tokens][Hq][D] bf16, boxes of [128 / G tokens][G
+// heads][64 elements] with 128-byte swizzle (one box per 64-column chunk of
+// a unit's Q tile).
 cudaError_t launch_prefill_umma(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                int head_dim, int block_size, int num_tokens, int num_sms, cudaStream_t stream);
+                                const CUtensorMap& tm_q, int head_dim, int block_size, int num_tokens, int num_sms,
+                                cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                               int head_dim, int block_size, int num_tokens, cudaStream_t stream);
 

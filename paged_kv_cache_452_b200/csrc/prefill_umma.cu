@@ -13,29 +13,35 @@
 // tile serves all of them.  One persistent CTA per SM walks its share of the
 // units; the rings, the S buffers and the barriers run on across units, so
 // the next unit's first tiles load while the current one finishes.
-//  * warps 0 and 18 walk the block table and bring the K and the V halves of
+//  * warps 0 and 6 walk the block table and bring the K and the V halves of
 //    128-key tiles into two rings of shared-memory stages with TMA (2-D
 //    boxes of [block][128 B], 128-byte swizzle, boxes of consecutive blocks
 //    stacked into one swizzled tile); a K stage is free again as soon as its
 //    S MMA has run, a V stage once its PV MMA has; blocks past the keys the
 //    unit needs are read out of range, which TMA fills with zeros; table
-//    entries are read one tile ahead;
+//    entries are read one tile ahead; the V loader also brings each unit's
+//    query rows into the Q tile with TMA (3-D boxes of [positions][group
+//    heads][128 B], which land in the MMA's row order) as soon as the
+//    previous unit's last S MMA has run, so the next unit's first S does not
+//    wait for a load issued after the previous unit's output;
 //  * warp 1 holds the TMEM allocation and, from one thread, issues
 //    S = Q K^T (M 128, N 128, K 16 steps; double-buffered S in TMEM) and
 //    O += P V (N = head_dim; O stays in TMEM across tiles; P read from
 //    TMEM), committing each to an mbarrier; the S two tiles ahead goes out
 //    as soon as the row warps have read a tile's S, its PV once its P is
 //    written;
-//  * warps 2..17 own a quarter of a query row per thread (four warps per
-//    TMEM lane quarter, so four per SM sub-partition to hide each tile's
-//    latencies): they read their 32 keys of the row of S from TMEM, mask
-//    (causal, context length), combine the row's max with the other quarters
-//    through shared memory, keep a running max reference that
-//    moves only when the row's max grows by more than 2^8 (then the row of
-//    O in TMEM and the running sum are rescaled: the result is unchanged,
-//    the rescale is rare), write P = 2^(s - ref) as bf16 into one of two P
-//    buffers in TMEM (so a tile's softmax need not wait for the previous
-//    tile's PV to finish reading its P), and at the end divide O by the sum.
+//  * warps 2..5 own one query row per thread (a warp per TMEM lane
+//    quarter, so one per SM sub-partition): they read the row's 128 scores
+//    of a tile from TMEM into registers, mask (causal, context length; only
+//    the tiles at a row's end), take the row's max, keep a running max
+//    reference that moves only when the row's max grows by more than 2^8
+//    (then the row of O in TMEM and the running sum are rescaled: the result
+//    is unchanged, the rescale is rare), write P = 2^(s - ref) as bf16 into
+//    one of two P buffers in TMEM (so a tile's softmax need not wait for the
+//    previous tile's PV to finish reading its P), and at the end divide O by
+//    the sum.  No row warp ever waits for another: each tile's exponentials
+//    (the SM's special-function units' 16 per clock) bound its time, close
+//    to the tensor pipe's time for the tile's two MMAs.
 // Every wait is bounded (2 s, then the error word is set); TMEM is freed on
 // every path.
 #include <cuda_runtime.h>
@@ -48,15 +54,20 @@ namespace {
 
 constexpr int kRows = 128;    // query rows per unit (positions x group): the MMA's M
 constexpr int kKeys = 128;    // keys per K/V tile: N of S = Q K^T, K of O = P V
-// Each query row is split into kParts parts (kKeys / kParts keys of every
-// tile, D / kParts columns of O), one thread per part: four row warps per
-// TMEM lane quarter, so every SM sub-partition runs four softmax warps.
-constexpr int kParts = 4;
+// Each query row may be split into kParts parts (kKeys / kParts keys of
+// every tile, D / kParts columns of O), one thread per part, the parts
+// combining the row's max and sum through shared memory.  One part: a thread
+// owns a whole row, its 128 scores of a tile in registers, and the row warps
+// never wait for one another (the exchange and its barrier cost more than
+// the extra warps hid).
+constexpr int kParts = 1;
 constexpr int kRowWarps = 4 * kParts;
 constexpr int kThreads = 32 * (kRowWarps + 3);  // warp 0 loads K, warp 1 issues MMAs, then the row warps, last loads V
 constexpr int kVWarp = kRowWarps + 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSmemOptIn = 232448;  // 227 KB per block
+constexpr int kSmemOptIn = 232448;  // 227 KB per block: dynamic plus static shared memory
+constexpr int kStaticSmem = 64;     // the kernel's static shared memory (warp_tot), at most
+static_assert(4 * (kThreads / 32) <= kStaticSmem, "static shared memory reserve");
 constexpr int kChunk = 128 * 128;   // one 128-byte-wide chunk of a 128-row tile
 constexpr float kRefSlack = 8.f;    // log2 growth of a row max before its reference moves
 constexpr int kUQ = 4;              // unit queue entries (the K loader claims, the other roles follow)
@@ -79,7 +90,7 @@ struct U {
 struct Bars {
   // kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], then s_full[2],
   // s_free[2], p_full[2], o_full[2], q_full, o_free, done, uq_full[kUQ],
-  // uq_empty[kUQ]
+  // uq_empty[kUQ], q_free
   uint64_t* kfull;
   uint64_t* kempty;
   uint64_t* vfull;
@@ -93,6 +104,7 @@ struct Bars {
   uint64_t* done;
   uint64_t* uq_full;
   uint64_t* uq_empty;
+  uint64_t* q_free;
 };
 
 struct ULayout {
@@ -108,13 +120,13 @@ __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int ns
   L.vring = off;
   off += (uint32_t)kvt * nsv;
   L.bars = off;
-  off += (uint32_t)(2 * nsk + 2 * nsv + 11 + 2 * kUQ) * 8;
+  off += (uint32_t)(2 * nsk + 2 * nsv + 12 + 2 * kUQ) * 8;
   L.tmem = off;
   off += 16;
   L.uq = off;  // unit queue [kUQ], then the row groups' unit slots [4 quarters][2]
   off += (kUQ + 8) * 4;
   L.xch = off;  // row max parts [2 tile parities][kParts][128 rows], row sum parts [kParts][128]
-  off += (2 * kParts * 128 + kParts * 128) * 4;
+  if (kParts > 1) off += (2 * kParts * 128 + kParts * 128) * 4;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
@@ -131,7 +143,7 @@ __device__ __forceinline__ uint32_t swz(int r, int u) { return (uint32_t)(r * 12
 template <int D, int BS, bool PFX>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_umma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        const PrefillParams p) {
+                        const __grid_constant__ CUtensorMap tm_q, const PrefillParams p) {
   using C = U<D, BS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -143,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* vring = smem + L.vring;
   uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* bx = bar0 + 2 * NSK + 2 * NSV;
-  Bars B{bar0, bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 6, bx + 8, bx + 9, bx + 10,
-         bx + 11, bx + 11 + kUQ};
+  Bars B{bar0,   bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 6, bx + 8, bx + 9,
+         bx + 10, bx + 11,   bx + 11 + kUQ,  bx + 11 + 2 * kUQ};
   int32_t* uq = reinterpret_cast<int32_t*>(smem + L.uq);
   int32_t* pair_idx = uq + kUQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem);
@@ -286,7 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&B.p_full[i], kRowWarps);
       dev::mbar_init(&B.o_full[i], 1);
     }
-    dev::mbar_init(B.q_full, kRowWarps);
+    // the Q tile: one TMA transaction (the V loader), or in the shared-prefix
+    // mode, whose rows are gathered member by member, one arrival per row warp
+    dev::mbar_init(B.q_full, PFX ? kRowWarps : 1);
+    dev::mbar_init(B.q_free, 1);
     dev::mbar_init(B.o_free, kRowWarps);
     dev::mbar_init(B.done, 1);
     for (int i = 0; i < kUQ; ++i) {
@@ -331,6 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     bool ok = true;
     int g = 0;
+    int st = 0;        // g % nsr
+    uint32_t lph = 0;  // (g / nsr) & 1
+    int qlast = -1;    // the last unit whose Q rows this warp loaded
+    const uint64_t qpol = dev::policy_evict_first();
     for (int n = 0;; ++n) {
       // queue entry n: the K loader claims the unit and publishes it, the V
       // loader reads it (a timed-out wait ends the walk, -1 for the others)
@@ -356,10 +375,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (idx < 0) break;
       const Unit u = unit_of(idx);
+      if constexpr (!PFX) {
+        if (is_v) {
+          // this unit's query rows, once the previous unit's S MMAs are done
+          // with the Q tile: rows first + q0 .. + QB - 1 (positions past the
+          // unit are other rows or zeros, masked by the row warps)
+          if (n > 0 && ok) ok = __all_sync(0xffffffffu, dev::mbar_wait(B.q_free, (uint32_t)((n - 1) & 1), p.err));
+          if (ok && lane == 0) {
+            dev::mbar_arrive_expect_tx(B.q_full, (uint32_t)C::QBYTES);
+#pragma unroll
+            for (int cq = 0; cq < C::NCH; ++cq)
+              dev::tma_load_3d(qs + cq * kChunk, &tm_q, cq * 64, u.h * G, u.first + u.q0, B.q_full, qpol);
+            qlast = n;
+          }
+          __syncwarp();
+          if (!ok) break;
+        }
+      }
       int32_t enext = entry(u, 0);
       for (int k = 0; k < u.ntiles && ok; ++k, ++g) {
-        const int st = g % nsr;
-        if (g >= nsr) ok = __all_sync(0xffffffffu, dev::mbar_wait(&emptyb[st], ((g / nsr) - 1) & 1, p.err));
+        if (g >= nsr) ok = __all_sync(0xffffffffu, dev::mbar_wait(&emptyb[st], lph ^ 1u, p.err));
         if (!ok) break;
         int32_t blk = enext;
         if (k + 1 < u.ntiles) enext = entry(u, k + 1);
@@ -375,13 +410,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane < C::BOXES)
           dev::tma_load_2d(ringb + (size_t)st * C::KVT + c * kChunk + j * BS * 128, tm, c * 64, y, &fullb[st], pol);
+        if (++st == nsr) {
+          st = 0;
+          lph ^= 1u;
+        }
       }
     }
-    // drain: the last stages issued must land before this CTA may exit
+    // drain: the last stages (and Q tile) issued must land before this CTA
+    // may exit
     if (lane == 0) {
       for (int d = max(0, g - nsr); d < g; ++d)
         dev::mbar_wait(&fullb[d % nsr], (uint32_t)((d / nsr) & 1), nullptr, 100000000ull);
+      if (qlast >= 0) dev::mbar_wait(B.q_full, (uint32_t)(qlast & 1), nullptr, 100000000ull);
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issue (one thread) ===========================
     if (lane == 0) {
@@ -392,19 +434,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = dev::umma_desc_sw128(dev::smem_u32(qs), 16, 1024);
       const uint64_t dk = dev::umma_desc_sw128(dev::smem_u32(kring), 16, 1024);
       const uint64_t dv = dev::umma_desc_sw128(dev::smem_u32(vring), kChunk, 1024);
+      // Ring stage and phase of the next S (K ring) and of the next PV (V
+      // ring), advanced tile by tile: this thread's path between MMAs is short
+      // and free of divisions, since every instruction on it delays the
+      // tensor pipe's next tile.
+      int ks_st = 0, vs_st = 0;
+      uint32_t ks_ph = 0, vs_ph = 0;
       // S[g & 1] = Q K_g^T once K_g has landed and S[g & 1]'s last reader is done
-      auto issue_s = [&](int g) -> bool {
-        if (!dev::mbar_wait(&B.kfull[g % NSK], (uint32_t)((g / NSK) & 1), p.err)) return false;
+      // `last`: the unit's last S, after which the Q tile may be reloaded
+      auto issue_s = [&](int g, bool last) -> bool {
+        if (!dev::mbar_wait(&B.kfull[ks_st], ks_ph, p.err)) return false;
         if (g >= 2 && !dev::mbar_wait(&B.s_free[g & 1], (uint32_t)(((g >> 1) - 1) & 1), p.err)) return false;
         dev::tc_fence_after();
-        const uint64_t kb = dk + (uint64_t)(((g % NSK) * C::KVT) >> 4);
+        const uint64_t kb = dk + (uint64_t)ks_st * (uint64_t)(C::KVT >> 4);
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS_S; ++ks) {
           const uint64_t off = (uint64_t)(((ks >> 2) * kChunk + (ks & 3) * 32) >> 4);
           dev::umma_ss(t_s0 + (uint32_t)((g & 1) * kKeys), dq + off, kb + off, idesc_s, ks > 0 ? 1u : 0u);
         }
         dev::umma_commit(&B.s_full[g & 1]);
-        dev::umma_commit(&B.kempty[g % NSK]);
+        dev::umma_commit(&B.kempty[ks_st]);
+        if (last) dev::umma_commit(B.q_free);
+        if (++ks_st == NSK) {
+          ks_st = 0;
+          ks_ph ^= 1u;
+        }
         return true;
       };
       bool ok = true;
@@ -418,24 +472,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (idx < 0) break;
         const Unit u = unit_of(idx);
         ok = dev::mbar_wait(B.q_full, (uint32_t)(nu & 1), p.err);  // this unit's Q rows are in place
-        if (ok && u.ntiles > 0) ok = issue_s(g0);
-        if (ok && u.ntiles > 1) ok = issue_s(g0 + 1);
+        if (ok && u.ntiles == 0) dev::umma_commit(B.q_free);
+        if (ok && u.ntiles > 0) ok = issue_s(g0, u.ntiles == 1);
+        if (ok && u.ntiles > 1) ok = issue_s(g0 + 1, u.ntiles == 2);
         for (int k = 0; k < u.ntiles && ok; ++k) {
           const int g = g0 + k;
           // S two tiles ahead goes out as soon as the row warps have read
           // S_g out of its buffer (early in tile g's softmax), so it has two
           // softmax durations to complete before they need it
-          if (k + 2 < u.ntiles) ok = issue_s(g + 2);
+          if (k + 2 < u.ntiles) ok = issue_s(g + 2, k + 3 == u.ntiles);
           if (!ok) break;
           // p_full[g & 1] and o_full[g & 1] complete once per tile of that
           // parity: tile g is their phase g >> 1
           ok = dev::mbar_wait(&B.p_full[g & 1], (uint32_t)((g >> 1) & 1), p.err) &&
-               dev::mbar_wait(&B.vfull[g % NSV], (uint32_t)((g / NSV) & 1), p.err);
+               dev::mbar_wait(&B.vfull[vs_st], vs_ph, p.err);
           // the previous unit's O has been read out before this unit overwrites it
           if (ok && k == 0 && nu > 0) ok = dev::mbar_wait(B.o_free, (uint32_t)((nu - 1) & 1), p.err);
           if (!ok) break;
           dev::tc_fence_after();
-          const uint64_t vb = dv + (uint64_t)(((g % NSV) * C::KVT) >> 4);
+          const uint64_t vb = dv + (uint64_t)vs_st * (uint64_t)(C::KVT >> 4);
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS_O; ++ks) {
             // A = P from TMEM buffer g & 1 (16 keys = 8 columns per step); B =
@@ -445,7 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                          vb + (uint64_t)((ks * 16 * 128) >> 4), idesc_o, (k > 0 || ks > 0) ? 1u : 0u);
           }
           dev::umma_commit(&B.o_full[g & 1]);
-          dev::umma_commit(&B.vempty[g % NSV]);
+          dev::umma_commit(&B.vempty[vs_st]);
+          if (++vs_st == NSV) {
+            vs_st = 0;
+            vs_ph ^= 1u;
+          }
         }
         g0 += u.ntiles;
       }
@@ -457,12 +516,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ======================= rows: softmax, P, output =========================
     // Thread = (row r, part hh): keys [HK hh, HK (hh+1)) of each tile and O
-    // columns [HD hh, HD (hh+1)).  The kParts warps of a lane quarter meet at
-    // named barrier 1 + quarter; they run the same units and tiles and pass
+    // columns [HD hh, HD (hh+1)).  With more than one part, the kParts warps of
+    // a lane quarter meet at named barrier 1 + quarter; they run the same units and tiles and pass
     // the same barriers even after a timed-out wait (then they skip the
     // remaining waits), so none can be left waiting.
     constexpr int HK = kKeys / kParts, HD = D / kParts;
-    static_assert(HK == 32 && (HD == 32 || HD == 16), "one TMEM load of S per part, one or half of O");
+    static_assert((HK == 32 || HK == 64 || HK == 128) && (HD == 16 || HD == 32 || HD == 64 || HD == 128),
+                  "one TMEM load of a part of S, one of a part of O");
     const int quarter = warp & 3, hh = (warp - 2) >> 2;
     const int r = 32 * quarter + lane;  // this thread's row (its TMEM lane)
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
@@ -478,21 +538,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0;; ++n) {
       // the group's first warp reads queue entry n and hands it to the others
       // through shared memory (two slots, alternating); all leave together
+      int idx = -1;
       {
         const int slot = n % kUQ;
         if (hh == 0) {
-          int idx = -1;
           wait_ok(&B.uq_full[slot], (uint32_t)((n / kUQ) & 1));
           if (ok) idx = uq[slot];
           __syncwarp();
           if (lane == 0) {
-            pair_idx[quarter * 2 + (n & 1)] = idx;
+            if constexpr (kParts > 1) pair_idx[quarter * 2 + (n & 1)] = idx;
             dev::mbar_arrive(&B.uq_empty[slot]);
           }
         }
-        dev::named_bar_sync(pair_bar, kGroup);
+        if constexpr (kParts > 1) {
+          dev::named_bar_sync(pair_bar, kGroup);
+          idx = pair_idx[quarter * 2 + (n & 1)];
+        }
       }
-      const int idx = pair_idx[quarter * 2 + (n & 1)];
       if (idx < 0) break;
       const Unit u = unit_of(idx);
       const bool valid = r < u.qn * G;
@@ -501,10 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // member slot first + r / G
       const int qrow = !PFX ? u.first + u.q0 + r / G : (valid ? __ldg(p.pfx_members + u.first + r / G) : 0);
       const int64_t grow = ((int64_t)qrow * hq + (int64_t)u.h * G + r % G) * D;
-      // ---- this part of the Q row into the swizzled Q tile (zero for rows
-      // past the unit); the previous unit's MMAs have all completed (its
-      // output was read after them)
-      {
+      // ---- shared-prefix mode: this part of the member's Q row into the
+      // swizzled Q tile (zero for rows past the unit); the previous unit's
+      // MMAs have all completed (its output was read after them)
+      if constexpr (PFX) {
         const uint4* src = reinterpret_cast<const uint4*>(p.q + grow * 2);
         constexpr int VU = C::NCH * 8 / kParts;  // 16-byte units of a part
 #pragma unroll
@@ -523,10 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::tc_fence_after();
         float sv[HK];
         {
-          uint32_t w[32];
-          dev::tmem_ld32(t_s0 + (uint32_t)((g & 1) * kKeys + HK * hh) + lane_addr, w);
+          uint32_t w[HK];
+          dev::tmem_ld(t_s0 + (uint32_t)((g & 1) * kKeys + HK * hh) + lane_addr, w);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(w[i]);
+          for (int i = 0; i < HK; ++i) sv[i] = __uint_as_float(w[i]);
         }
         dev::tc_fence_before();
         __syncwarp();
@@ -534,20 +596,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // mask; this part's max, then the row's (the scale is positive, so
         // it is applied to the max and folded into the exponent's FMA)
         const int lim = min(pos + 1, u.seq_len) - k * kKeys - HK * hh;  // keys [0, lim) of this part are visible
-        float mp[4];
+        if (!valid || lim < HK) {  // only the tiles at a row's causal or context end
 #pragma unroll
-        for (int i = 0; i < 4; ++i) mp[i] = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < HK; ++i) {
-          sv[i] = (valid && i < lim) ? sv[i] : -INFINITY;
-          mp[i & 3] = fmaxf(mp[i & 3], sv[i]);
+          for (int i = 0; i < HK; ++i) sv[i] = (valid && i < lim) ? sv[i] : -INFINITY;
         }
-        const float mh = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-        xmax[((g & 1) * kParts + hh) * 128 + r] = mh;
-        dev::named_bar_sync(pair_bar, kGroup);
-        float mrow = mh;
+        float mp[8];
 #pragma unroll
-        for (int q2 = 0; q2 < kParts; ++q2) mrow = fmaxf(mrow, xmax[((g & 1) * kParts + q2) * 128 + r]);
+        for (int i = 0; i < 8; ++i) mp[i] = sv[i];
+#pragma unroll
+        for (int i = 8; i < HK; ++i) mp[i & 7] = fmaxf(mp[i & 7], sv[i]);
+        float mrow = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                           fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        if constexpr (kParts > 1) {
+          xmax[((g & 1) * kParts + hh) * 128 + r] = mrow;
+          dev::named_bar_sync(pair_bar, kGroup);
+#pragma unroll
+          for (int q2 = 0; q2 < kParts; ++q2) mrow = fmaxf(mrow, xmax[((g & 1) * kParts + q2) * 128 + r]);
+        }
         const float mx = mrow * p.scale_log2;
         const bool move = mx > ref + kRefSlack;
         const float alpha = move ? dev::ex2(ref - mx) : 1.f;
@@ -558,17 +623,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P = 2^(s * scale - ref) as bf16 pairs, in registers: this work
         // overlaps the previous tile's PV MMA
         uint32_t pk[HK / 2];
-        float sp[4];
+        float sp[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) sp[i] = 0.f;
+        for (int i = 0; i < 8; ++i) sp[i] = 0.f;
 #pragma unroll
         for (int i = 0; i < HK / 2; ++i) {
           const float a = dev::ex2(fmaf(sv[2 * i], p.scale_log2, -ref));
           const float b = dev::ex2(fmaf(sv[2 * i + 1], p.scale_log2, -ref));
-          sp[i & 3] += a + b;
+          sp[i & 7] += a + b;
           pk[i] = dev::pack_bf16(a, b);
         }
-        lsum += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+        lsum += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
         // a rescale needs O stable: the previous tile's PV has finished
         if (k > 0 && __any_sync(0xffffffffu, move)) {
           wait_ok(&B.o_full[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1));
@@ -578,10 +643,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // reference use 1)
             const uint32_t ta = t_o + (uint32_t)(HD * hh) + lane_addr;
             uint32_t w[HD];
-            if constexpr (HD == 32) dev::tmem_ld32(ta, w); else dev::tmem_ld16(ta, w);
+            dev::tmem_ld(ta, w);
 #pragma unroll
             for (int i = 0; i < HD; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-            if constexpr (HD == 32) dev::tmem_st32(ta, w); else dev::tmem_st16(ta, w);
+            dev::tmem_st(ta, w);
           }
         }
         // P buffer g & 1 was last read by the PV of tile g - 2 (an earlier
@@ -591,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           dev::tc_fence_after();
         }
         // this part's HK keys, two per column, into P buffer g & 1
-        dev::tmem_st16(t_p + (uint32_t)((g & 1) * (kKeys / 2) + (HK / 2) * hh) + lane_addr, pk);
+        dev::tmem_st(t_p + (uint32_t)((g & 1) * (kKeys / 2) + (HK / 2) * hh) + lane_addr, pk);
         // the tile holding the context's end: slots past it hold stale pool
         // bytes (masked scores, but 0 * NaN would poison P V): zero their V rows
         const int key0 = k * kKeys;
@@ -615,14 +680,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u.ntiles > 0) {
         wait_ok(&B.o_full[(g0 + u.ntiles - 1) & 1], (uint32_t)(((g0 + u.ntiles - 1) >> 1) & 1));
         dev::tc_fence_after();
-        xsum[hh * 128 + r] = lsum;
-        dev::named_bar_sync(pair_bar, kGroup);
-        float total = 0.f;
+        float total = lsum;
+        if constexpr (kParts > 1) {
+          xsum[hh * 128 + r] = lsum;
+          dev::named_bar_sync(pair_bar, kGroup);
+          total = 0.f;
 #pragma unroll
-        for (int q2 = 0; q2 < kParts; ++q2) total += xsum[q2 * 128 + r];
+          for (int q2 = 0; q2 < kParts; ++q2) total += xsum[q2 * 128 + r];
+        }
         uint32_t w[HD];
-        if constexpr (HD == 32) dev::tmem_ld32(t_o + (uint32_t)(HD * hh) + lane_addr, w);
-        else dev::tmem_ld16(t_o + (uint32_t)(HD * hh) + lane_addr, w);
+        dev::tmem_ld(t_o + (uint32_t)(HD * hh) + lane_addr, w);
         if constexpr (PFX) {
           // partial row of member slot first + r / G, q head h * G + r % G:
           // (max reference, sum) and this part of the unnormalised O
@@ -670,7 +737,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int BS, bool PFX = false>
-cudaError_t launch_u(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v, int grid,
+cudaError_t launch_u(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_q,
+                     int grid,
                      cudaStream_t stream) {
   using C = U<D, BS>;
   const ULayout L = u_layout(C::QBYTES, C::KVT, p.nstages, p.nstages_v, p.rows.num_seqs);
@@ -694,7 +762,7 @@ cudaError_t launch_u(const PrefillParams& p, const CUtensorMap& tm_k, const CUte
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_k, tm_v, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm_k, tm_v, tm_q, p);
 }
 
 }  // namespace
@@ -705,12 +773,12 @@ bool prefill_umma_supported(int kv, int q, int head_dim, int block_size, int gro
 }
 
 cudaError_t launch_prefill_umma(const PrefillParams& p_in, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                int head_dim, int block_size, int num_tokens, int num_sms, cudaStream_t stream) {
+                                const CUtensorMap& tm_q, int head_dim, int block_size, int num_tokens, int num_sms, cudaStream_t stream) {
   PrefillParams p = p_in;
   const int nch = head_dim / 64;
   const int qbytes = nch * kChunk, kvt = nch * kChunk;
   const int fixed = (int)u_layout(qbytes, kvt, 0, 0, p.rows.num_seqs).total;
-  const int nbuf = (kSmemOptIn - fixed) / (kvt + 16);  // K and V stages that fit
+  const int nbuf = (kSmemOptIn - kStaticSmem - fixed) / (kvt + 16);  // K and V stages that fit
   const int nsk = min(4, nbuf / 2), nsv = min(4, nbuf - nbuf / 2);
   if (nsk < 2 || nsv < 2) return cudaErrorNotSupported;  // too many sequences for the unit table: caller falls back
   p.nstages = nsk;
@@ -719,10 +787,10 @@ cudaError_t launch_prefill_umma(const PrefillParams& p_in, const CUtensorMap& tm
   const int64_t bound = ((int64_t)num_tokens / qb + p.rows.num_seqs) * p.num_kv_heads;  // units, at most
   if (bound <= 0) return cudaSuccess;
   const int64_t grid = bound < num_sms ? bound : num_sms;  // one persistent CTA per SM
-  if (head_dim == 128 && block_size == 16) return launch_u<128, 16>(p, tm_k, tm_v, (int)grid, stream);
-  if (head_dim == 128 && block_size == 32) return launch_u<128, 32>(p, tm_k, tm_v, (int)grid, stream);
-  if (head_dim == 64 && block_size == 16) return launch_u<64, 16>(p, tm_k, tm_v, (int)grid, stream);
-  if (head_dim == 64 && block_size == 32) return launch_u<64, 32>(p, tm_k, tm_v, (int)grid, stream);
+  if (head_dim == 128 && block_size == 16) return launch_u<128, 16>(p, tm_k, tm_v, tm_q, (int)grid, stream);
+  if (head_dim == 128 && block_size == 32) return launch_u<128, 32>(p, tm_k, tm_v, tm_q, (int)grid, stream);
+  if (head_dim == 64 && block_size == 16) return launch_u<64, 16>(p, tm_k, tm_v, tm_q, (int)grid, stream);
+  if (head_dim == 64 && block_size == 32) return launch_u<64, 32>(p, tm_k, tm_v, tm_q, (int)grid, stream);
   return cudaErrorNotSupported;
 }
 
@@ -732,7 +800,7 @@ cudaError_t launch_prefix_umma(const PrefillParams& p_in, const CUtensorMap& tm_
   const int nch = head_dim / 64;
   const int qbytes = nch * kChunk, kvt = nch * kChunk;
   const int fixed = (int)u_layout(qbytes, kvt, 0, 0, p.rows.num_seqs).total;
-  const int nbuf = (kSmemOptIn - fixed) / (kvt + 16);
+  const int nbuf = (kSmemOptIn - kStaticSmem - fixed) / (kvt + 16);
   const int nsk = min(4, nbuf / 2), nsv = min(4, nbuf - nbuf / 2);
   if (nsk < 2 || nsv < 2) return cudaErrorNotSupported;
   p.nstages = nsk;
@@ -744,10 +812,10 @@ cudaError_t launch_prefix_umma(const PrefillParams& p_in, const CUtensorMap& tm_
   const int64_t bound = ((int64_t)p.num_members / qb + p.rows.num_seqs) * chunks * p.num_kv_heads;
   if (bound <= 0) return cudaSuccess;
   const int64_t grid = bound < num_sms ? bound : num_sms;
-  if (head_dim == 128 && block_size == 16) return launch_u<128, 16, true>(p, tm_k, tm_v, (int)grid, stream);
-  if (head_dim == 128 && block_size == 32) return launch_u<128, 32, true>(p, tm_k, tm_v, (int)grid, stream);
-  if (head_dim == 64 && block_size == 16) return launch_u<64, 16, true>(p, tm_k, tm_v, (int)grid, stream);
-  if (head_dim == 64 && block_size == 32) return launch_u<64, 32, true>(p, tm_k, tm_v, (int)grid, stream);
+  if (head_dim == 128 && block_size == 16) return launch_u<128, 16, true>(p, tm_k, tm_v, tm_k, (int)grid, stream);
+  if (head_dim == 128 && block_size == 32) return launch_u<128, 32, true>(p, tm_k, tm_v, tm_k, (int)grid, stream);
+  if (head_dim == 64 && block_size == 16) return launch_u<64, 16, true>(p, tm_k, tm_v, tm_k, (int)grid, stream);
+  if (head_dim == 64 && block_size == 32) return launch_u<64, 32, true>(p, tm_k, tm_v, tm_k, (int)grid, stream);
   return cudaErrorNotSupported;
 }
 
