@@ -25,11 +25,13 @@
 //    previous unit's last S MMA has run, so the next unit's first S does not
 //    wait for a load issued after the previous unit's output;
 //  * warp 1 holds the TMEM allocation and, from one thread, issues
-//    S = Q K^T (M 128, N 128, K 16 steps; double-buffered S in TMEM) and
-//    O += P V (N = head_dim; O stays in TMEM across tiles; P read from
-//    TMEM), committing each to an mbarrier; the S two tiles ahead goes out
-//    as soon as the row warps have read a tile's S, its PV once its P is
-//    written;
+//    S = Q K^T (M 128, N 128, K 16 steps; double-buffered S in TMEM), each
+//    as soon as its K tile has landed and the row warps have read the S two
+//    tiles back; warp 7, from one thread, issues O += P V (N = head_dim; O
+//    stays in TMEM across tiles; P read from TMEM) once a tile's P is
+//    written; each thread commits its MMAs to mbarriers.  The two streams
+//    share no TMEM and wait for different things, so neither thread's waits
+//    hold up the other's MMAs;
 //  * warps 2..5 own one query row per thread (a warp per TMEM lane
 //    quarter, so one per SM sub-partition): they read the row's 128 scores
 //    of a tile from TMEM into registers, mask (causal, context length; only
@@ -62,8 +64,11 @@ constexpr int kKeys = 128;    // keys per K/V tile: N of S = Q K^T, K of O = P V
 // the extra warps hid).
 constexpr int kParts = 1;
 constexpr int kRowWarps = 4 * kParts;
-constexpr int kThreads = 32 * (kRowWarps + 3);  // warp 0 loads K, warp 1 issues MMAs, then the row warps, last loads V
+// warp 0 loads K, warp 1 issues the S MMAs, then the row warps, then the V
+// loader and the warp that issues the PV MMAs
+constexpr int kThreads = 32 * (kRowWarps + 4);
 constexpr int kVWarp = kRowWarps + 2;
+constexpr int kPvWarp = kRowWarps + 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemOptIn = 232448;  // 227 KB per block: dynamic plus static shared memory
 constexpr int kStaticSmem = 64;     // the kernel's static shared memory (warp_tot), at most
@@ -71,9 +76,10 @@ static_assert(4 * (kThreads / 32) <= kStaticSmem, "static shared memory reserve"
 constexpr int kChunk = 128 * 128;   // one 128-byte-wide chunk of a 128-row tile
 constexpr float kRefSlack = 8.f;    // log2 growth of a row max before its reference moves
 constexpr int kUQ = 4;              // unit queue entries (the K loader claims, the other roles follow)
-// roles that read each queue entry: the V loader, the MMA thread and one
-// warp of each of the four row-warp groups (one group per TMEM lane quarter)
-constexpr int kUQReaders = 6;
+// roles that read each queue entry: the V loader, the two MMA threads and
+// one warp of each of the four row-warp groups (one group per TMEM lane
+// quarter)
+constexpr int kUQReaders = 7;
 
 template <int D, int BS>
 struct U {
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::mbar_init(B.q_full, PFX ? kRowWarps : 1);
     dev::mbar_init(B.q_free, 1);
     dev::mbar_init(B.o_free, kRowWarps);
-    dev::mbar_init(B.done, 1);
+    dev::mbar_init(B.done, 2);
     for (int i = 0; i < kUQ; ++i) {
       dev::mbar_init(&B.uq_full[i], 1);
       dev::mbar_init(&B.uq_empty[i], kUQReaders);
@@ -424,8 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (qlast >= 0) dev::mbar_wait(B.q_full, (uint32_t)(qlast & 1), nullptr, 100000000ull);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ======================= MMA issue (one thread) ===========================
+  } else if (warp == 1 || warp == kPvWarp) {
+    // ============ MMA issue: S (warp 1) or PV (warp 7), one thread each =========
+    const bool is_pv = warp == kPvWarp;
     if (lane == 0) {
       const uint32_t idesc_s = dev::umma_idesc_bf16(kKeys, false);
       const uint32_t idesc_o = dev::umma_idesc_bf16(D, true);
@@ -434,10 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = dev::umma_desc_sw128(dev::smem_u32(qs), 16, 1024);
       const uint64_t dk = dev::umma_desc_sw128(dev::smem_u32(kring), 16, 1024);
       const uint64_t dv = dev::umma_desc_sw128(dev::smem_u32(vring), kChunk, 1024);
-      // Ring stage and phase of the next S (K ring) and of the next PV (V
-      // ring), advanced tile by tile: this thread's path between MMAs is short
-      // and free of divisions, since every instruction on it delays the
-      // tensor pipe's next tile.
+      // Ring stage and phase of the next S (K ring) or the next PV (V ring),
+      // advanced tile by tile: the issuing path between MMAs is kept short and
+      // free of divisions, since every instruction on it delays the tensor
+      // pipe's next tile.
       int ks_st = 0, vs_st = 0;
       uint32_t ks_ph = 0, vs_ph = 0;
       // S[g & 1] = Q K_g^T once K_g has landed and S[g & 1]'s last reader is done
@@ -471,17 +478,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::mbar_arrive(&B.uq_empty[slot]);
         if (idx < 0) break;
         const Unit u = unit_of(idx);
-        ok = dev::mbar_wait(B.q_full, (uint32_t)(nu & 1), p.err);  // this unit's Q rows are in place
-        if (ok && u.ntiles == 0) dev::umma_commit(B.q_free);
-        if (ok && u.ntiles > 0) ok = issue_s(g0, u.ntiles == 1);
-        if (ok && u.ntiles > 1) ok = issue_s(g0 + 1, u.ntiles == 2);
+        if (!is_pv) {
+          // S of every tile of the unit, each as early as its inputs allow
+          // (two tiles ahead of the row warps at most: the S buffers)
+          ok = dev::mbar_wait(B.q_full, (uint32_t)(nu & 1), p.err);  // this unit's Q rows are in place
+          if (ok && u.ntiles == 0) dev::umma_commit(B.q_free);
+          for (int k = 0; k < u.ntiles && ok; ++k) ok = issue_s(g0 + k, k + 1 == u.ntiles);
+          g0 += u.ntiles;
+          continue;
+        }
         for (int k = 0; k < u.ntiles && ok; ++k) {
           const int g = g0 + k;
-          // S two tiles ahead goes out as soon as the row warps have read
-          // S_g out of its buffer (early in tile g's softmax), so it has two
-          // softmax durations to complete before they need it
-          if (k + 2 < u.ntiles) ok = issue_s(g + 2, k + 3 == u.ntiles);
-          if (!ok) break;
           // p_full[g & 1] and o_full[g & 1] complete once per tile of that
           // parity: tile g is their phase g >> 1
           ok = dev::mbar_wait(&B.p_full[g & 1], (uint32_t)((g >> 1) & 1), p.err) &&
@@ -508,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         g0 += u.ntiles;
       }
-      // every MMA issued above has completed before TMEM may be freed
+      // every MMA this thread issued has completed before TMEM may be freed
+      // (the barrier takes one commit from each of the two threads)
       dev::umma_commit(B.done);
       dev::mbar_wait(B.done, 0, nullptr, 100000000ull);
     }
