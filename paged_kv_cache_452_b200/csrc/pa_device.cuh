@@ -293,6 +293,11 @@ __device__ __forceinline__ void tmem_st(uint32_t a, const uint32_t (&r)[32]) { t
 __device__ __forceinline__ void tmem_st(uint32_t a, const uint32_t (&r)[64]) { tmem_st64(a, r); }
 __device__ __forceinline__ void tmem_st(uint32_t a, const uint32_t (&r)[128]) { tmem_st128(a, r); }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 // ---- conversions -------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -612,9 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) mp[i] = sv[i];
 #pragma unroll
-        for (int i = 8; i < HK; ++i) mp[i & 7] = fmaxf(mp[i & 7], sv[i]);
-        float mrow = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                           fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        for (int i = 8; i < HK; i += 2) mp[(i >> 1) & 7] = dev::max3(mp[(i >> 1) & 7], sv[i], sv[i + 1]);
+        float mrow = dev::max3(dev::max3(mp[0], mp[1], mp[2]), dev::max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
         if constexpr (kParts > 1) {
           xmax[((g & 1) * kParts + hh) * 128 + r] = mrow;
           dev::named_bar_sync(pair_bar, kGroup);
@@ -678,8 +677,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(vt + (rest >> 3) * kChunk + key * 128 + (rest & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         dev::tc_fence_before();
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(&B.p_full[g & 1]);
