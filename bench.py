@@ -529,7 +529,7 @@ def e2e_measure(m, device, args, world):
     return {"ms_per_step": e2e_ms, "h2d_bytes_per_step": off, "d2h_bytes_per_step": d2h, "output_matches": same}
 
 
-PER_CONFIG = ("prefix_bf16", "fp8_long", "mixed_prefill_bs16", "mixed_prefill_bs32")
+PER_CONFIG = ("prefix_bf16", "fp8_long", "mixed_prefill_bs16", "mixed_prefill_bs32", "long_prefix_bf16")
 
 
 def bench_ours(args):

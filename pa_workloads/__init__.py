@@ -23,6 +23,11 @@ Workloads (sizes as named by the paged-attention benchmark plan):
 * ``mixed_prefill``: 8 prefill chunks of 512 query tokens over 0..4096 prior
   tokens each, plus 248 decode rows over contexts uniform in [64, 4096];
   32/8 heads, head_dim 128, block 16 or 32.
+* ``long_prefix_bf16`` (a case of our own for the shared-prefix path, not
+  one of the plan's five): 64 sequences that all share one 32768-token
+  prefix (2048 blocks, 134 MB of K/V, more than the L2 cache holds), suffix
+  lengths lognormal (median 512, sigma 1) clipped to [16, 2048]; 32/8 heads,
+  head_dim 128, block 16.
 
 Each has a ``small`` variant with the same structure at sizes a plain CPU
 oracle finishes in seconds.  Randomness: ``tiny_fp32`` draws everything from
@@ -267,6 +272,18 @@ def prefix_bf16(size: str = "full") -> Workload:
                    32, 8, 128, 16, ctx, np.ones(n), prefix_len=prefix, sharing=sharing)
 
 
+def long_prefix_bf16(size: str = "full") -> Workload:
+    key = 5 if size == "full" else 105
+    if size == "full":
+        n, prefix, median, lo, hi = 64, 32768, 512, 16, 2048
+    else:
+        n, prefix, median, lo, hi = 6, 320, 40, 16, 120
+    suf = rng(key, GLOBAL, S_SUFFIX).lognormal(mean=np.log(median), sigma=1.0, size=n)
+    suf = np.clip(np.rint(suf), lo, hi).astype(np.int64)
+    return _finish("long_prefix_bf16" + ("" if size == "full" else "_small"), key, "bf16", "bf16",
+                   32, 8, 128, 16, suf + prefix, np.ones(n), prefix_len=prefix, sharing=np.ones(n, dtype=bool))
+
+
 def fp8_long(size: str = "full") -> Workload:
     key = 3 if size == "full" else 103
     n, lo, hi = (128, 4096, 32768) if size == "full" else (4, 100, 700)
@@ -333,6 +350,7 @@ WORKLOADS = {
     "fp8_long": fp8_long,
     "mixed_prefill_bs16": lambda size="full": mixed_prefill(16, size),
     "mixed_prefill_bs32": lambda size="full": mixed_prefill(32, size),
+    "long_prefix_bf16": long_prefix_bf16,
 }
 
 

@@ -214,8 +214,14 @@ bool prefix_path(const pa_cache_desc* d) {
 }
 
 // Bytes of the prefix partials after pa_decode's own scratch.
+int prefix_chunk_keys_for(const pa_cache_desc* d, int32_t num_members, int32_t max_prefix_blocks) {
+  return prefix_chunk_keys(max_prefix_blocks, d->block_size, num_members, d->num_q_heads / d->num_kv_heads,
+                           d->num_kv_heads);
+}
+
 size_t prefix_partial_bytes(const pa_cache_desc* d, int32_t num_members, int32_t max_prefix_blocks, size_t* ml_bytes) {
-  const size_t chunks = ((size_t)max_prefix_blocks * d->block_size + kPrefixChunkKeys - 1) / kPrefixChunkKeys;
+  const size_t ck = (size_t)prefix_chunk_keys_for(d, num_members, max_prefix_blocks);
+  const size_t chunks = ((size_t)max_prefix_blocks * d->block_size + ck - 1) / ck;
   const size_t rows = chunks * (size_t)num_members * d->num_q_heads;
   *ml_bytes = (rows * 2 * 4 + 255) / 256 * 256;
   return *ml_bytes + rows * d->head_dim * 4;
@@ -229,6 +235,7 @@ struct PrefixArgs {
   const float* ml;
   const float* o;
   int32_t num_members;
+  int32_t chunk_keys;
 };
 
 // The new tokens' rows that pa_decode_fused writes in the decode launch.
@@ -296,7 +303,7 @@ int run_decode_tc(const pa_cache_desc* d, const void* q, const void* k_cache, co
     p.pfx_ml = pa->ml;
     p.pfx_o = pa->o;
     p.pfx_members = pa->num_members;
-    p.pfx_chunk_blocks = kPrefixChunkKeys / d->block_size;
+    p.pfx_chunk_blocks = pa->chunk_keys / d->block_size;
   }
   if (fw) {
     p.k_new = static_cast<const uint8_t*>(fw->k_new);
@@ -546,7 +553,7 @@ int pa_decode_prefix(const pa_cache_desc* d, const void* q, const void* k_cache,
   pp.pfx_members = prefix_members;
   pp.pfx_blocks = prefix_blocks;
   pp.num_members = num_members;
-  pp.chunk_keys = kPrefixChunkKeys;
+  pp.chunk_keys = prefix_chunk_keys_for(d, num_members, max_prefix_blocks);
   pp.pfx_ml = pml;
   pp.pfx_o = po;
   cudaError_t e = launch_prefix_umma(pp, tm_k, tm_v, d->head_dim, d->block_size, sms, st);
@@ -555,7 +562,7 @@ int pa_decode_prefix(const pa_cache_desc* d, const void* q, const void* k_cache,
                      workspace, workspace_bytes, stream);
   if ((rc = cuda_status(e, who))) return rc;
   // 2. the suffixes on the decode kernel, folding each member's chunk partials
-  const PrefixArgs pa{seq_prefix, seq_slot, prefix_blocks, pml, po, num_members};
+  const PrefixArgs pa{seq_prefix, seq_slot, prefix_blocks, pml, po, num_members, pp.chunk_keys};
   return run_decode_tc(d, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, nullptr, num_seqs,
                        num_seqs, scale, out, workspace, base, st, who, nullptr, &pa);
 }

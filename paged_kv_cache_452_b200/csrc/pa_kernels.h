@@ -87,7 +87,7 @@ struct DecodeParams {
   const float* pfx_ml;  // [chunks][num_members][Hq][2]
   const float* pfx_o;   // [chunks][num_members][Hq][D]
   int32_t pfx_members;
-  int32_t pfx_chunk_blocks;  // blocks per chunk (kPrefixChunkKeys / block_size)
+  int32_t pfx_chunk_blocks;  // blocks per prefix chunk (prefix_chunk_keys / block_size)
   DecodeWorkspace ws;
 };
 
@@ -128,8 +128,26 @@ struct PrefillParams {
   float* pfx_o;                // [chunks][M][Hq][D]
 };
 
-// The split of a prefix into chunks of keys that pa_decode_prefix uses.
-constexpr int kPrefixChunkKeys = 256;
+// The split of a prefix into chunks of keys that pa_decode_prefix uses: a
+// unit of the prefix kernel is (prefix, kv head, 128 / G members, chunk).
+// Chunks are whole 128-key tiles, at least two, and as few as give about
+// kPrefixUnits units in all: every chunk adds a partial per member row that
+// the prefix kernel writes and the decode folds in one after the other, and
+// measured on B200 that fold outweighs spreading the prefix over more SMs
+// (a 32768-token prefix shared by 64 sequences: 91 us at about 128 units,
+// 131 us at 512; a 1024-token prefix: 194 us with 256-key chunks, 237 us
+// with 128).  A function of the batch's sizes alone, so the workspace size
+// does not depend on the device.
+constexpr int kPrefixUnits = 128;
+inline int prefix_chunk_keys(int max_prefix_blocks, int block_size, int num_members, int group, int num_kv_heads) {
+  const long long keys = (long long)max_prefix_blocks * block_size;
+  const int per_tile = 128 / group;  // members per unit
+  const long long member_tiles = num_members > per_tile ? (num_members + per_tile - 1) / per_tile : 1;
+  const long long per_chunk = member_tiles * (num_kv_heads > 0 ? num_kv_heads : 1);
+  const long long chunks = per_chunk >= kPrefixUnits ? 1 : (kPrefixUnits + per_chunk - 1) / per_chunk;
+  const long long ck = ((keys + chunks - 1) / chunks + 127) / 128 * 128;
+  return (int)(ck < 256 ? 256 : ck);
+}
 cudaError_t launch_prefix_umma(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                int head_dim, int block_size, int num_sms, cudaStream_t stream);
 bool prefill_tc_supported(int kv, int q, int head_dim, int block_size, int group);

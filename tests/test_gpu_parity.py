@@ -87,7 +87,8 @@ def run_and_check(wl, device, seqs=None):
     return b, err
 
 
-SMALL = ["tiny_fp32", "gqa_bf16", "prefix_bf16", "fp8_long", "mixed_prefill_bs16", "mixed_prefill_bs32"]
+SMALL = ["tiny_fp32", "gqa_bf16", "prefix_bf16", "fp8_long", "mixed_prefill_bs16", "mixed_prefill_bs32",
+         "long_prefix_bf16"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -277,7 +278,7 @@ def test_bad_table_entry_in_prompt_rows_is_flagged(cuda_device):
 
 
 FULL = [("gqa_bf16", None), ("prefix_bf16", [0, 1, 2, 127, 128, 129, 200, 255]), ("fp8_long", [0, 77]),
-        ("mixed_prefill_bs16", [0, 7, 8, 100, 255]), ("mixed_prefill_bs32", [3, 100])]
+        ("mixed_prefill_bs16", [0, 7, 8, 100, 255]), ("mixed_prefill_bs32", [3, 100]), ("long_prefix_bf16", [0, 63])]
 
 
 @pytest.mark.slow

@@ -39,6 +39,8 @@ def _groups_case(name, n_groups, members, prefix_len, suffix_hi, private, seed=0
 
 CASES = {
     "prefix_bf16": lambda: W.make("prefix_bf16", "small"),
+    # every sequence shares the prefix: one prefix of 20 blocks, chunks of 256 + 64 keys
+    "long_prefix_bf16": lambda: W.make("long_prefix_bf16", "small"),
     # 3 member tiles of 32 (group 4), a 20-block prefix: chunks of 256 + 64 keys
     "many_members": lambda: _groups_case("many_members", 1, 80, 320, 300, 10, num_q_heads=32, num_kv_heads=8),
     "two_prefixes": lambda: _groups_case("two_prefixes", 2, 7, 96, 150, 5, seed=1),

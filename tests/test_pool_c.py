@@ -126,7 +126,7 @@ def test_random_traces_match_model(seed):
 
 
 @pytest.mark.parametrize("name", ["tiny_fp32", "gqa_bf16", "prefix_bf16", "fp8_long", "mixed_prefill_bs16",
-                                  "mixed_prefill_bs32"])
+                                  "mixed_prefill_bs32", "long_prefix_bf16"])
 @pytest.mark.parametrize("size", ["small", "full"])
 def test_workload_admission_matches_model(name, size):
     wl = W.make(name, size)
