@@ -35,15 +35,14 @@
 //  * warps 2..5 own one query row per thread (a warp per TMEM lane
 //    quarter, so one per SM sub-partition): they read the row's 128 scores
 //    of a tile from TMEM into registers, mask (causal, context length; only
-//    the tiles at a row's end), take the row's max, keep a running max
-//    reference that moves only when the row's max grows by more than 2^8
-//    (then the row of O in TMEM and the running sum are rescaled: the result
-//    is unchanged, the rescale is rare), write P = 2^(s - ref) as bf16 into
-//    one of two P buffers in TMEM (so a tile's softmax need not wait for the
+//    the tiles at a row's end), write P = 2^(s - ref) as bf16 into one of
+//    two P buffers in TMEM (so a tile's softmax need not wait for the
 //    previous tile's PV to finish reading its P), and at the end divide O by
-//    the sum.  No row warp ever waits for another: each tile's exponentials
-//    (the SM's special-function units' 16 per clock) bound its time, close
-//    to the tensor pipe's time for the tile's two MMAs.
+//    the sum.  The exponent reference ref is the row max of the unit's first
+//    tile; later tiles skip the max unless their weights would grow past
+//    2^64 (then ref moves and O and the running sum are rescaled: rare, and
+//    the result is the same softmax up to rounding).  No row warp waits
+//    for another; their softmax sets the tile period.
 // Every wait is bounded (2 s, then the error word is set); TMEM is freed on
 // every path.
 #include <cuda_runtime.h>
@@ -56,14 +55,11 @@ namespace {
 
 constexpr int kRows = 128;    // query rows per unit (positions x group): the MMA's M
 constexpr int kKeys = 128;    // keys per K/V tile: N of S = Q K^T, K of O = P V
-// Each query row may be split into kParts parts (kKeys / kParts keys of
-// every tile, D / kParts columns of O), one thread per part, the parts
-// combining the row's max and sum through shared memory.  One part: a thread
-// owns a whole row, its 128 scores of a tile in registers, and the row warps
-// never wait for one another (the exchange and its barrier cost more than
-// the extra warps hid).
-constexpr int kParts = 1;
-constexpr int kRowWarps = 4 * kParts;
+// One softmax warp per TMEM lane quarter, a thread per query row: the row's
+// 128 scores of a tile sit in registers and no row warp waits for another
+// (splitting a row over two or four warps that exchange row maxima through
+// shared memory measured slower).
+constexpr int kRowWarps = 4;
 // warp 0 loads K, warp 1 issues the S MMAs, then the row warps, then the V
 // loader and the warp that issues the PV MMAs
 constexpr int kThreads = 32 * (kRowWarps + 4);
@@ -74,11 +70,10 @@ constexpr int kSmemOptIn = 232448;  // 227 KB per block: dynamic plus static sha
 constexpr int kStaticSmem = 64;     // the kernel's static shared memory (warp_tot), at most
 static_assert(4 * (kThreads / 32) <= kStaticSmem, "static shared memory reserve");
 constexpr int kChunk = 128 * 128;   // one 128-byte-wide chunk of a 128-row tile
-constexpr float kRefSlack = 8.f;    // log2 growth of a row max before its reference moves
+constexpr float kBig = 18446744073709551616.f;  // 2^64: the most a tile's weights may sum to on the fast path
 constexpr int kUQ = 4;              // unit queue entries (the K loader claims, the other roles follow)
 // roles that read each queue entry: the V loader, the two MMA threads and
-// one warp of each of the four row-warp groups (one group per TMEM lane
-// quarter)
+// the four row warps
 constexpr int kUQReaders = 7;
 
 template <int D, int BS>
@@ -114,7 +109,7 @@ struct Bars {
 };
 
 struct ULayout {
-  uint32_t q, kring, vring, bars, tmem, uq, xch, prefix, total;
+  uint32_t q, kring, vring, bars, tmem, uq, prefix, total;
 };
 __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int nsv, int num_seqs) {
   ULayout L;
@@ -129,10 +124,8 @@ __host__ __device__ inline ULayout u_layout(int qbytes, int kvt, int nsk, int ns
   off += (uint32_t)(2 * nsk + 2 * nsv + 12 + 2 * kUQ) * 8;
   L.tmem = off;
   off += 16;
-  L.uq = off;  // unit queue [kUQ], then the row groups' unit slots [4 quarters][2]
-  off += (kUQ + 8) * 4;
-  L.xch = off;  // row max parts [2 tile parities][kParts][128 rows], row sum parts [kParts][128]
-  if (kParts > 1) off += (2 * kParts * 128 + kParts * 128) * 4;
+  L.uq = off;  // unit queue [kUQ]
+  off += kUQ * 4;
   L.prefix = off;
   off += (uint32_t)(num_seqs + 1) * 4;
   L.total = off + 1024;  // slack for aligning the base to 1024 bytes
@@ -164,7 +157,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars B{bar0,   bar0 + NSK, bar0 + 2 * NSK, bar0 + 2 * NSK + NSV, bx, bx + 2, bx + 4, bx + 6, bx + 8, bx + 9,
          bx + 10, bx + 11,   bx + 11 + kUQ,  bx + 11 + 2 * kUQ};
   int32_t* uq = reinterpret_cast<int32_t*>(smem + L.uq);
-  int32_t* pair_idx = uq + kUQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem);
   int32_t* prefix = reinterpret_cast<int32_t*>(smem + L.prefix);  // units before sequence s
   __shared__ int32_t warp_tot[kThreads / 32];
@@ -523,45 +515,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ======================= rows: softmax, P, output =========================
-    // Thread = (row r, part hh): keys [HK hh, HK (hh+1)) of each tile and O
-    // columns [HD hh, HD (hh+1)).  With more than one part, the kParts warps of
-    // a lane quarter meet at named barrier 1 + quarter; they run the same units and tiles and pass
-    // the same barriers even after a timed-out wait (then they skip the
-    // remaining waits), so none can be left waiting.
-    constexpr int HK = kKeys / kParts, HD = D / kParts;
-    static_assert((HK == 32 || HK == 64 || HK == 128) && (HD == 16 || HD == 32 || HD == 64 || HD == 128),
-                  "one TMEM load of a part of S, one of a part of O");
-    const int quarter = warp & 3, hh = (warp - 2) >> 2;
+    // Thread = row r (its TMEM lane): the row's 128 keys of each tile and its
+    // D columns of O.  The exponent reference of a row is taken from the
+    // unit's first tile (its row max); later tiles keep it and skip the max,
+    // since 2^(s * scale - ref) only has to stay finite: fp32 and bf16 share
+    // an exponent range up to 2^127, so a tile whose sum of weights stays at
+    // most kBig (2^64) is exact to rounding.  A tile above that (or not
+    // finite) takes the slow path: its row max, a new reference, the running
+    // sum and O rescaled, and the tile's weights recomputed.
+    const int quarter = warp & 3;
     const int r = 32 * quarter + lane;  // this thread's row (its TMEM lane)
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
-    const int pair_bar = 1 + quarter;
-    constexpr int kGroup = 32 * kParts;                     // threads at a quarter's named barrier
-    float* xmax = reinterpret_cast<float*>(smem + L.xch);  // [tile parity][part][row]
-    float* xsum = xmax + 2 * kParts * 128;                  // [part][row]
     bool ok = true;
     auto wait_ok = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(0xffffffffu, dev::mbar_wait(bar, parity, p.err));
     };
+    // the row's scores of a tile, keys past `lim` (or all, for a row past the
+    // unit) set to -inf
+    auto load_s = [&](uint32_t ts, float (&sv)[kKeys], bool whole, int lim, bool valid) {
+      uint32_t w[kKeys];
+      dev::tmem_ld(ts, w);
+#pragma unroll
+      for (int i = 0; i < kKeys; ++i) sv[i] = __uint_as_float(w[i]);
+      if (!whole) {  // only the tiles at a row's causal or context end
+#pragma unroll
+        for (int i = 0; i < kKeys; ++i) sv[i] = (valid && i < lim) ? sv[i] : -INFINITY;
+      }
+    };
+    // the row's max score times the scale (the scale is positive)
+    auto row_max = [&](const float (&sv)[kKeys]) {
+      float mp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mp[i] = sv[i];
+#pragma unroll
+      for (int i = 8; i < kKeys; i += 2) mp[(i >> 1) & 7] = dev::max3(mp[(i >> 1) & 7], sv[i], sv[i + 1]);
+      return dev::max3(dev::max3(mp[0], mp[1], mp[2]), dev::max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) *
+             p.scale_log2;
+    };
+    // P = 2^(s * scale - ref) as bf16 pairs, and the tile's fp32 sum of them
+    auto weights = [&](const float (&sv)[kKeys], float ref, uint32_t (&pk)[kKeys / 2]) {
+      float sp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sp[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kKeys / 2; ++i) {
+        const float a = dev::ex2(fmaf(sv[2 * i], p.scale_log2, -ref));
+        const float b = dev::ex2(fmaf(sv[2 * i + 1], p.scale_log2, -ref));
+        sp[i & 7] += a + b;
+        pk[i] = dev::pack_bf16(a, b);
+      }
+      return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+    };
     int g0 = 0;
     for (int n = 0;; ++n) {
-      // the group's first warp reads queue entry n and hands it to the others
-      // through shared memory (two slots, alternating); all leave together
+      // each row warp reads queue entry n itself
       int idx = -1;
       {
         const int slot = n % kUQ;
-        if (hh == 0) {
-          wait_ok(&B.uq_full[slot], (uint32_t)((n / kUQ) & 1));
-          if (ok) idx = uq[slot];
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (kParts > 1) pair_idx[quarter * 2 + (n & 1)] = idx;
-            dev::mbar_arrive(&B.uq_empty[slot]);
-          }
-        }
-        if constexpr (kParts > 1) {
-          dev::named_bar_sync(pair_bar, kGroup);
-          idx = pair_idx[quarter * 2 + (n & 1)];
-        }
+        wait_ok(&B.uq_full[slot], (uint32_t)((n / kUQ) & 1));
+        if (ok) idx = uq[slot];
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&B.uq_empty[slot]);
       }
       if (idx < 0) break;
       const Unit u = unit_of(idx);
@@ -571,14 +585,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // member slot first + r / G
       const int qrow = !PFX ? u.first + u.q0 + r / G : (valid ? __ldg(p.pfx_members + u.first + r / G) : 0);
       const int64_t grow = ((int64_t)qrow * hq + (int64_t)u.h * G + r % G) * D;
-      // ---- shared-prefix mode: this part of the member's Q row into the
-      // swizzled Q tile (zero for rows past the unit); the previous unit's
-      // MMAs have all completed (its output was read after them)
+      // ---- shared-prefix mode: the member's Q row into the swizzled Q tile
+      // (zero for rows past the unit); the previous unit's MMAs have all
+      // completed (its output was read after them)
       if constexpr (PFX) {
         const uint4* src = reinterpret_cast<const uint4*>(p.q + grow * 2);
-        constexpr int VU = C::NCH * 8 / kParts;  // 16-byte units of a part
 #pragma unroll
-        for (int v = hh * VU; v < (hh + 1) * VU; ++v) {
+        for (int v = 0; v < C::NCH * 8; ++v) {
           const uint4 x = valid ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
           *reinterpret_cast<uint4*>(qs + (v >> 3) * kChunk + swz(r, v & 7)) = x;
         }
@@ -586,84 +599,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(B.q_full);
       }
-      float ref = -1e30f, lsum = 0.f;
+      float ref = -1e30f, lsum = 0.f;  // a row with nothing visible keeps -1e30: its weights are 0
       for (int k = 0; k < u.ntiles; ++k) {
         const int g = g0 + k;
         wait_ok(&B.s_full[g & 1], (uint32_t)((g >> 1) & 1));
         dev::tc_fence_after();
-        float sv[HK];
-        {
-          uint32_t w[HK];
-          dev::tmem_ld(t_s0 + (uint32_t)((g & 1) * kKeys + HK * hh) + lane_addr, w);
+        const uint32_t ts = t_s0 + (uint32_t)((g & 1) * kKeys) + lane_addr;
+        const int lim = min(pos + 1, u.seq_len) - k * kKeys;  // keys [0, lim) of the tile are visible
+        const bool whole = valid && lim >= kKeys;
+        float sv[kKeys];
+        load_s(ts, sv, whole, lim, valid);
+        if (k == 0) ref = fmaxf(ref, row_max(sv));
+        uint32_t pk[kKeys / 2];
+        float tsum = weights(sv, ref, pk);
+        if (k > 0 && __any_sync(0xffffffffu, !(tsum <= kBig))) {
+          // slow path (the S buffer is still this tile's: it is released below)
+          load_s(ts, sv, whole, lim, valid);
+          const float mx = row_max(sv);
+          const bool move = mx > ref;
+          const float alpha = move ? dev::ex2(ref - mx) : 1.f;
+          if (move) {
+            lsum *= alpha;
+            ref = mx;
+          }
+          tsum = weights(sv, ref, pk);
+          // O rescaled once the previous tile's PV has finished (rows that keep
+          // their reference use 1)
+          wait_ok(&B.o_full[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1));
+          dev::tc_fence_after();
+          uint32_t w[D];
+          dev::tmem_ld(t_o + lane_addr, w);
 #pragma unroll
-          for (int i = 0; i < HK; ++i) sv[i] = __uint_as_float(w[i]);
+          for (int i = 0; i < D; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+          dev::tmem_st(t_o + lane_addr, w);
         }
+        lsum += tsum;
+        // S buffer g & 1 is free for the S two tiles on
         dev::tc_fence_before();
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(&B.s_free[g & 1]);
-        // mask; this part's max, then the row's (the scale is positive, so
-        // it is applied to the max and folded into the exponent's FMA)
-        const int lim = min(pos + 1, u.seq_len) - k * kKeys - HK * hh;  // keys [0, lim) of this part are visible
-        if (!valid || lim < HK) {  // only the tiles at a row's causal or context end
-#pragma unroll
-          for (int i = 0; i < HK; ++i) sv[i] = (valid && i < lim) ? sv[i] : -INFINITY;
-        }
-        float mp[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mp[i] = sv[i];
-#pragma unroll
-        for (int i = 8; i < HK; i += 2) mp[(i >> 1) & 7] = dev::max3(mp[(i >> 1) & 7], sv[i], sv[i + 1]);
-        float mrow = dev::max3(dev::max3(mp[0], mp[1], mp[2]), dev::max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
-        if constexpr (kParts > 1) {
-          xmax[((g & 1) * kParts + hh) * 128 + r] = mrow;
-          dev::named_bar_sync(pair_bar, kGroup);
-#pragma unroll
-          for (int q2 = 0; q2 < kParts; ++q2) mrow = fmaxf(mrow, xmax[((g & 1) * kParts + q2) * 128 + r]);
-        }
-        const float mx = mrow * p.scale_log2;
-        const bool move = mx > ref + kRefSlack;
-        const float alpha = move ? dev::ex2(ref - mx) : 1.f;
-        if (move) {
-          lsum *= alpha;
-          ref = mx;
-        }
-        // P = 2^(s * scale - ref) as bf16 pairs, in registers: this work
-        // overlaps the previous tile's PV MMA
-        uint32_t pk[HK / 2];
-        float sp[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sp[i] = 0.f;
-#pragma unroll
-        for (int i = 0; i < HK / 2; ++i) {
-          const float a = dev::ex2(fmaf(sv[2 * i], p.scale_log2, -ref));
-          const float b = dev::ex2(fmaf(sv[2 * i + 1], p.scale_log2, -ref));
-          sp[i & 7] += a + b;
-          pk[i] = dev::pack_bf16(a, b);
-        }
-        lsum += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-        // a rescale needs O stable: the previous tile's PV has finished
-        if (k > 0 && __any_sync(0xffffffffu, move)) {
-          wait_ok(&B.o_full[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1));
-          dev::tc_fence_after();
-          {
-            // rescale this row's part of O in TMEM (rows that keep their
-            // reference use 1)
-            const uint32_t ta = t_o + (uint32_t)(HD * hh) + lane_addr;
-            uint32_t w[HD];
-            dev::tmem_ld(ta, w);
-#pragma unroll
-            for (int i = 0; i < HD; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-            dev::tmem_st(ta, w);
-          }
-        }
         // P buffer g & 1 was last read by the PV of tile g - 2 (an earlier
         // unit's PVs are all done: its epilogue waited for them)
         if (k >= 2) {
           wait_ok(&B.o_full[g & 1], (uint32_t)(((g >> 1) - 1) & 1));
           dev::tc_fence_after();
         }
-        // this part's HK keys, two per column, into P buffer g & 1
-        dev::tmem_st(t_p + (uint32_t)((g & 1) * (kKeys / 2) + (HK / 2) * hh) + lane_addr, pk);
+        // the row's 128 keys, two per column, into P buffer g & 1
+        dev::tmem_st(t_p + (uint32_t)((g & 1) * (kKeys / 2)) + lane_addr, pk);
         // the tile holding the context's end: slots past it hold stale pool
         // bytes (masked scores, but 0 * NaN would poison P V): zero their V rows
         const int key0 = k * kKeys;
@@ -683,45 +665,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(&B.p_full[g & 1]);
       }
-      // ---- O / sum -> this part of the output row; then O is free ----
+      // ---- O / sum -> the output row; then O is free ----
       if (u.ntiles > 0) {
         wait_ok(&B.o_full[(g0 + u.ntiles - 1) & 1], (uint32_t)(((g0 + u.ntiles - 1) >> 1) & 1));
         dev::tc_fence_after();
-        float total = lsum;
-        if constexpr (kParts > 1) {
-          xsum[hh * 128 + r] = lsum;
-          dev::named_bar_sync(pair_bar, kGroup);
-          total = 0.f;
-#pragma unroll
-          for (int q2 = 0; q2 < kParts; ++q2) total += xsum[q2 * 128 + r];
-        }
-        uint32_t w[HD];
-        dev::tmem_ld(t_o + (uint32_t)(HD * hh) + lane_addr, w);
+        uint32_t w[D];
+        dev::tmem_ld(t_o + lane_addr, w);
         if constexpr (PFX) {
           // partial row of member slot first + r / G, q head h * G + r % G:
-          // (max reference, sum) and this part of the unnormalised O
+          // (reference, sum) and the unnormalised O
           const int64_t prow =
               ((int64_t)u.chunk * p.num_members + u.first + r / G) * hq + (int64_t)u.h * G + r % G;
-          if (valid && ok && hh == 0) *reinterpret_cast<float2*>(p.pfx_ml + prow * 2) = make_float2(ref, total);
-          float4* dst = reinterpret_cast<float4*>(p.pfx_o + prow * D + HD * hh);
+          if (valid && ok) *reinterpret_cast<float2*>(p.pfx_ml + prow * 2) = make_float2(ref, lsum);
+          float4* dst = reinterpret_cast<float4*>(p.pfx_o + prow * D);
           if (valid && ok) {
 #pragma unroll
-            for (int uu = 0; uu < HD / 4; ++uu)
+            for (int uu = 0; uu < D / 4; ++uu)
               dst[uu] = make_float4(__uint_as_float(w[4 * uu]), __uint_as_float(w[4 * uu + 1]),
                                     __uint_as_float(w[4 * uu + 2]), __uint_as_float(w[4 * uu + 3]));
           }
         } else {
-          const float inv = valid ? 1.f / total : 0.f;
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (grow + HD * hh) * 2);
+          const float inv = valid ? 1.f / lsum : 0.f;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + grow * 2);
           if (valid && ok) {
 #pragma unroll
-            for (int uu = 0; uu < HD / 8; ++uu) {
-              uint32_t pk[4];
+            for (int uu = 0; uu < D / 8; ++uu) {
+              uint32_t pq[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                pk[e] = dev::pack_bf16(__uint_as_float(w[8 * uu + 2 * e]) * inv,
+                pq[e] = dev::pack_bf16(__uint_as_float(w[8 * uu + 2 * e]) * inv,
                                        __uint_as_float(w[8 * uu + 2 * e + 1]) * inv);
-              dst[uu] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[uu] = make_uint4(pq[0], pq[1], pq[2], pq[3]);
             }
           }
         }
