@@ -91,6 +91,44 @@ SMALL = ["tiny_fp32", "gqa_bf16", "prefix_bf16", "fp8_long", "mixed_prefill_bs16
          "long_prefix_bf16"]
 
 
+def outscoring_draws(wl, late_from, factor, seed=5):
+    """Seeded N(0,1) draws for wl, keys of the cached context from position
+    late_from on scaled by `factor`: scores there exceed the first 128 keys'
+    by far more than 2^64 in the weights, so the tcgen05 prompt-row kernel's
+    rows take their slow path (the reference moves, O and the sum are
+    rescaled).  Sequences with equal prefix_group values share their first
+    wl.prefix_len tokens' draws."""
+    g = np.random.default_rng(seed)
+    hkv, hq, d = wl.num_kv_heads, wl.num_q_heads, wl.head_dim
+    shared = {}
+    ks, vs = [], []
+    for s in range(wl.num_seqs):
+        n = int(wl.context_lens[s])
+        k = g.standard_normal((n, hkv, d), dtype=np.float32)
+        v = g.standard_normal((n, hkv, d), dtype=np.float32)
+        grp = int(wl.prefix_group[s]) if wl.prefix_group is not None else -1
+        if grp >= 0:
+            if grp not in shared:
+                shared[grp] = (k[:wl.prefix_len].copy(), v[:wl.prefix_len].copy())
+            k[:wl.prefix_len], v[:wl.prefix_len] = shared[grp]
+        k[late_from:] *= factor
+        ks.append(k)
+        vs.append(v)
+    t = wl.num_new_tokens
+    wl._fixed = {"k": ks, "v": vs, "k_new": g.standard_normal((t, hkv, d), dtype=np.float32),
+                 "v_new": g.standard_normal((t, hkv, d), dtype=np.float32),
+                 "q": g.standard_normal((t, hq, d), dtype=np.float32)}
+    return wl
+
+
+def test_prompt_rows_whose_later_keys_outscore_the_first_tile(cuda_device):
+    # sequence 0: 64 prompt rows over 300 cached tokens, keys 200.. scaled;
+    # sequence 1: 130 prompt rows over 40 cached tokens (unscaled)
+    wl = outscoring_draws(W.custom("outscore", context_lens=[300, 40], q_lens=[64, 130], num_q_heads=8,
+                                   num_kv_heads=2), late_from=200, factor=48.0)
+    run_and_check(wl, cuda_device)
+
+
 @pytest.mark.parametrize("name", SMALL)
 def test_workload_small(name, cuda_device):
     run_and_check(W.make(name, "small"), cuda_device)

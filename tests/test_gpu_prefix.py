@@ -85,6 +85,23 @@ def test_prefix_decode_matches_oracle(name, cuda_device):
         assert torch.equal(rows, rows[:1].expand_as(rows))
 
 
+def test_prefix_chunk_whose_later_keys_outscore_its_first_tile(cuda_device):
+    """The shared-prefix kernel's rows take the slow path inside a chunk: a
+    640-token prefix (chunks of 256 keys), keys 160.. scaled."""
+    from test_gpu_parity import outscoring_draws
+    wl = outscoring_draws(W.custom("outscore_prefix", context_lens=[700, 660, 720, 645], num_q_heads=8,
+                                   num_kv_heads=2, prefix_len=640, prefix_group=[0, 0, 0, 0]),
+                          late_from=160, factor=48.0)
+    b, plan = _run(wl, cuda_device)
+    assert plan.groups.num_prefixes == 1
+    assert pa.workspace_error(plan.workspace) == 0
+    exp = expected(wl)
+    out = b.out.detach().cpu().double().numpy()[exp["rows"]]
+    assert np.isfinite(out).all()
+    err = float(np.abs(out - exp["out"]).max())
+    assert err <= TOL, f"max abs error {err}"
+
+
 def test_prefix_decode_replayed_from_a_graph(cuda_device):
     wl = CASES["many_members"]()
     b, plan = _run(wl, cuda_device)
