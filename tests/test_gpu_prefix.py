@@ -146,12 +146,17 @@ def test_prefix_longer_than_a_context_is_flagged(cuda_device):
 
 
 @pytest.mark.slow
-def test_prefix_decode_full_size_sampled(cuda_device):
-    wl = W.make("prefix_bf16", "full")
+@pytest.mark.parametrize("name,members,seqs", [
+    ("prefix_bf16", 128, [0, 1, 63, 127, 128, 200, 255]),
+    # a 32768-token prefix: eight chunks of 4096 keys (32-tile units), folded
+    # eight deep into every member's suffix
+    ("long_prefix_bf16", 64, [0, 31, 63]),
+])
+def test_prefix_decode_full_size_sampled(name, members, seqs, cuda_device):
+    wl = W.make(name, "full")
     b, plan = _run(wl, cuda_device)
-    assert plan.groups.num_prefixes == 1 and plan.groups.num_members == 128
+    assert plan.groups.num_prefixes == 1 and plan.groups.num_members == members
     assert pa.workspace_error(plan.workspace) == 0
-    seqs = [0, 1, 63, 127, 128, 200, 255]
     exp = expected(wl, seqs)
     out = b.out.detach().cpu().double().numpy()[exp["rows"]]
     err = float(np.abs(out - exp["out"]).max())
